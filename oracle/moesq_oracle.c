@@ -1,0 +1,401 @@
+/*
+ * Oracle for the paired-4:8 NVFP4 MoE expert path.  TEST INFRASTRUCTURE ONLY:
+ * nothing on the product path may link, load or call this file; only the
+ * tests, the smoke check and the benchmark's CPU-baseline leg do.
+ *
+ * Plain, slow, single-threaded C written from the definitions in
+ * "Hardware-Native Joint Sparse-Quantization for Trillion-Scale
+ * Mixture-of-Experts" (arXiv 2610.02241) and the model card
+ * "Kimi-K2.5-P48NVFP4-MoESQ".  Every function names the passage it follows.
+ * It shares no source with the CUDA library.  Floating point that decides an
+ * integer (a scale code, a value code, a kept pair) is done in IEEE binary32
+ * with one rounding per operation, in the order written (build with
+ * -ffp-contract=off so that no multiply-add is fused).  Sums that produce
+ * real outputs are done in binary64.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------ codecs */
+
+/* E2M1 value grid {0, +-0.5, +-1, +-1.5, +-2, +-3, +-4, +-6} (paper, App. A,
+ * Fig. 3 caption).  Code assignment: bit 3 is the sign, the three low bits
+ * index the magnitudes in increasing order (OCP Microscaling spec, E2M1). */
+static const double E2M1_MAG[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+double oracle_e2m1_value(int code) {
+    double m = E2M1_MAG[code & 7];
+    return (code & 8) ? -m : m;
+}
+
+/* Nearest-neighbour projection onto the E2M1 grid (paper, Sec. 3.2, Eq. 3:
+ * Pi_G).  Brute force over the 8 magnitudes; an exact tie goes to the even
+ * code; |x| above 6 lands on 6.  A result of magnitude 0 is always +0 (code 0).
+ * x must not be NaN. */
+int oracle_e2m1_encode(float x) {
+    double a = fabs((double)x);
+    int best = 0;
+    double bestd = a;                         /* distance to magnitude 0 */
+    for (int c = 1; c < 8; ++c) {
+        double d = fabs(a - E2M1_MAG[c]);
+        if (d < bestd || (d == bestd && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            bestd = d;
+        }
+    }
+    if (best == 0) return 0;
+    return (x < 0.0f) ? (best | 8) : best;
+}
+
+/* Unsigned E4M3 (paper: "UE4M3", max 448, Sec. 3.4 Eq. 5): exponent bias 7,
+ * 3 mantissa bits, subnormals m * 2^-9, code 0x7F is not a number. */
+double oracle_ue4m3_value(int code) {
+    int e = (code >> 3) & 15, m = code & 7;
+    if ((code & 0x7F) == 0x7F) return NAN;
+    if (e == 0) return ldexp((double)m, -9);
+    return ldexp(1.0 + m / 8.0, e - 7);
+}
+
+/* Pi_E4M3 of Eq. 5 for x >= 0: the nearest code, an exact tie to the even
+ * mantissa (even code), values above 448 onto 448.  Codes 0..126 are
+ * increasing in value, so a binary search finds the neighbours. */
+int oracle_ue4m3_encode(float x) {
+    double a = (double)x;
+    if (!(a > 0.0)) return 0;
+    if (a >= 448.0) return 0x7E;
+    int lo = 0, hi = 0x7E;                    /* value(lo) <= a < value(hi) */
+    while (hi - lo > 1) {
+        int mid = (lo + hi) / 2;
+        if (oracle_ue4m3_value(mid) <= a) lo = mid; else hi = mid;
+    }
+    double dl = a - oracle_ue4m3_value(lo), dh = oracle_ue4m3_value(hi) - a;
+    if (dl < dh) return lo;
+    if (dh < dl) return hi;
+    return (lo & 1) ? hi : lo;
+}
+
+static float bf16_to_float(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+/* Round to nearest even on the bit pattern; inputs are finite. */
+static uint16_t double_to_bf16(double v) {
+    float f = (float)v;
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
+}
+
+uint16_t oracle_bf16_round(double v) { return double_to_bf16(v); }
+
+/* ---------------------------------------------------- NVFP4 scale rule (Eq. 5)
+ * gamma = 448 / (max_b ||Y_b||_inf / 6); a zero tensor gets gamma = 1. */
+float oracle_global_scale(float amax_t) {
+    if (!(amax_t > 0.0f)) return 1.0f;
+    volatile float t = amax_t / 6.0f;
+    return 448.0f / t;
+}
+
+/* One 32-element block (16 kept values for weights, 32 for activations):
+ * code_b = Pi_E4M3(gamma * amax_b / 6); s_b = value(code_b) / gamma (Eq. 5);
+ * each value becomes Pi_G(v / s_b) (Eq. 3).  A block whose scale code is 0
+ * has s_b = 0 and dequantises to 0 whatever its codes, so its codes are 0. */
+static int block_scale_code(float gamma, float amax_b) {
+    volatile float p = gamma * amax_b;
+    volatile float sc = p / 6.0f;
+    return oracle_ue4m3_encode(sc);
+}
+
+static int quantize_value(float v, int scode, float gamma) {
+    if (scode == 0) return 0;
+    volatile float s_b = (float)oracle_ue4m3_value(scode) / gamma;
+    volatile float q = v / s_b;
+    return oracle_e2m1_encode(q);
+}
+
+/* --------------------------------------------------------- weight packing
+ * Paired 4:8 support (paper, Sec. 3.2 and App. A Eq. 6: six patterns per 8
+ * weights, each keeps two of the four adjacent pairs; model card: "exactly 2
+ * pairs are kept").  The kept pairs of a group are its two pairs of largest
+ * squared L2 norm (w0^2 + w1^2, binary32), an exact tie keeping the lower pair
+ * index.  Scales are then computed on the masked tensor (paper, Sec. 3.4:
+ * select the pattern, recompute the final scales, pack).
+ *
+ * Storage (model card, "pair-bitmask v1"): values [M][K/4] = the two kept
+ * bytes of every 4-byte chunk in K order, one byte = one pair, low nibble =
+ * the even K element; mask [M][K/16], 4 bits per chunk (bit p = pair p kept),
+ * low nibble = lower-K chunk; scales [M][K/32] UE4M3 codes; gamma = Eq. 5's
+ * tensor multiplier. */
+static void select_pairs(const float *w8, int kept[4]) {
+    float score[4];
+    for (int p = 0; p < 4; ++p) {
+        volatile float a = w8[2 * p] * w8[2 * p];
+        volatile float b = w8[2 * p + 1] * w8[2 * p + 1];
+        score[p] = a + b;
+    }
+    /* rank of pair p = number of pairs that beat it */
+    for (int p = 0; p < 4; ++p) {
+        int beaten = 0;
+        for (int q = 0; q < 4; ++q)
+            if (q != p && (score[q] > score[p] || (score[q] == score[p] && q < p))) ++beaten;
+        kept[p] = beaten < 2;
+    }
+}
+
+void oracle_pack_weights(const uint16_t *w_bf16, int M, int K,
+                         uint8_t *values, uint8_t *mask, uint8_t *scales, float *gamma_out) {
+    float *wm = (float *)malloc(sizeof(float) * (size_t)K);   /* masked row */
+    uint8_t *keep = (uint8_t *)malloc((size_t)K / 8);          /* 4-bit kept set per group */
+    float amax_t = 0.0f;
+    /* pass 1: support and tensor amax of the kept values */
+    for (int m = 0; m < M; ++m) {
+        for (int k = 0; k < K; ++k) wm[k] = bf16_to_float(w_bf16[(size_t)m * K + k]);
+        for (int g = 0; g < K / 8; ++g) {
+            int kept[4];
+            select_pairs(wm + 8 * g, kept);
+            for (int p = 0; p < 4; ++p)
+                if (kept[p])
+                    for (int i = 0; i < 2; ++i) {
+                        float a = fabsf(wm[8 * g + 2 * p + i]);
+                        if (a > amax_t) amax_t = a;
+                    }
+        }
+    }
+    float gamma = oracle_global_scale(amax_t);
+    *gamma_out = gamma;
+    /* pass 2: block scales, value codes, storage bytes */
+    for (int m = 0; m < M; ++m) {
+        for (int k = 0; k < K; ++k) wm[k] = bf16_to_float(w_bf16[(size_t)m * K + k]);
+        for (int g = 0; g < K / 8; ++g) {
+            int kept[4], bits = 0;
+            select_pairs(wm + 8 * g, kept);
+            for (int p = 0; p < 4; ++p) {
+                if (kept[p]) bits |= 1 << p;
+                else wm[8 * g + 2 * p] = wm[8 * g + 2 * p + 1] = 0.0f;
+            }
+            keep[g] = (uint8_t)bits;
+        }
+        for (int b = 0; b < K / 32; ++b) {
+            float amax_b = 0.0f;
+            for (int i = 0; i < 32; ++i) {
+                float a = fabsf(wm[32 * b + i]);
+                if (a > amax_b) amax_b = a;
+            }
+            int sc = block_scale_code(gamma, amax_b);
+            scales[(size_t)m * (K / 32) + b] = (uint8_t)sc;
+            for (int gg = 0; gg < 4; ++gg) {
+                int g = 4 * b + gg, slot = 0;
+                for (int p = 0; p < 4; ++p) {
+                    if (!(keep[g] >> p & 1)) continue;
+                    int c0 = quantize_value(wm[8 * g + 2 * p], sc, gamma);
+                    int c1 = quantize_value(wm[8 * g + 2 * p + 1], sc, gamma);
+                    values[(size_t)m * (K / 4) + 2 * g + slot] = (uint8_t)(c0 | (c1 << 4));
+                    ++slot;
+                }
+            }
+        }
+        for (int j = 0; j < K / 16; ++j)
+            mask[(size_t)m * (K / 16) + j] = (uint8_t)(keep[2 * j] | (keep[2 * j + 1] << 4));
+    }
+    free(wm);
+    free(keep);
+}
+
+/* Dense reconstruction of the packed weight (dequantised, pruned positions
+ * zero): W~[m][k] = value(code) * value(scale) / gamma. */
+void oracle_unpack_weights(const uint8_t *values, const uint8_t *mask, const uint8_t *scales,
+                           float gamma, int M, int K, double *w_out) {
+    for (int m = 0; m < M; ++m) {
+        for (int g = 0; g < K / 8; ++g) {
+            int bits = (mask[(size_t)m * (K / 16) + g / 2] >> (4 * (g & 1))) & 15;
+            int slot = 0;
+            double s = oracle_ue4m3_value(scales[(size_t)m * (K / 32) + g / 4]);
+            for (int p = 0; p < 4; ++p) {
+                double v0 = 0.0, v1 = 0.0;
+                if (bits >> p & 1) {
+                    int byte = values[(size_t)m * (K / 4) + 2 * g + slot];
+                    v0 = oracle_e2m1_value(byte & 15) * s / (double)gamma;
+                    v1 = oracle_e2m1_value(byte >> 4) * s / (double)gamma;
+                    ++slot;
+                }
+                w_out[(size_t)m * K + 8 * g + 2 * p] = v0;
+                w_out[(size_t)m * K + 8 * g + 2 * p + 1] = v1;
+            }
+        }
+    }
+}
+
+/* -------------------------------------------------- activation quantiser
+ * Q_a (paper, Sec. 3.3-3.4 and App. D.1; model card "Activations": NVFP4,
+ * dynamic per-32 group scales, a float32 global scale stored per expert
+ * linear): each row's 32-element blocks get Eq. 5's block scale under the
+ * given gamma; codes [rows][K/2] (low nibble = even k), scales [rows][K/32]. */
+void oracle_quantize_rows(const float *x, int rows, int K, float gamma,
+                          uint8_t *codes, uint8_t *scales) {
+    for (int r = 0; r < rows; ++r) {
+        const float *xr = x + (size_t)r * K;
+        for (int b = 0; b < K / 32; ++b) {
+            float amax_b = 0.0f;
+            for (int i = 0; i < 32; ++i) {
+                float a = fabsf(xr[32 * b + i]);
+                if (a > amax_b) amax_b = a;
+            }
+            int sc = block_scale_code(gamma, amax_b);
+            scales[(size_t)r * (K / 32) + b] = (uint8_t)sc;
+            for (int i = 0; i < 16; ++i) {
+                int c0 = quantize_value(xr[32 * b + 2 * i], sc, gamma);
+                int c1 = quantize_value(xr[32 * b + 2 * i + 1], sc, gamma);
+                codes[(size_t)r * (K / 2) + 16 * b + i] = (uint8_t)(c0 | (c1 << 4));
+            }
+        }
+    }
+}
+
+void oracle_quantize_rows_bf16(const uint16_t *x_bf16, int rows, int K, float gamma,
+                               uint8_t *codes, uint8_t *scales) {
+    float *xf = (float *)malloc(sizeof(float) * (size_t)K);
+    for (int r = 0; r < rows; ++r) {
+        for (int k = 0; k < K; ++k) xf[k] = bf16_to_float(x_bf16[(size_t)r * K + k]);
+        oracle_quantize_rows(xf, 1, K, gamma, codes + (size_t)r * (K / 2), scales + (size_t)r * (K / 32));
+    }
+    free(xf);
+}
+
+/* Largest |x| over a bf16 tensor, then Eq. 5's gamma: the static activation
+ * global scale calibrated on a batch. */
+float oracle_act_global_scale(const uint16_t *x_bf16, long long n) {
+    float amax = 0.0f;
+    for (long long i = 0; i < n; ++i) {
+        float a = fabsf(bf16_to_float(x_bf16[i]));
+        if (a > amax) amax = a;
+    }
+    return oracle_global_scale(amax);
+}
+
+/* ---------------------------------------------------------------- routing
+ * Top-k routing with softmax gate weights (the pages keep vLLM's routing;
+ * the workloads use softmax top-k).  Selection by descending logit, an exact
+ * tie to the lower expert index; weights are the softmax over all E experts
+ * (binary32, max subtracted, no renormalisation over the k chosen).
+ * Tokens are then grouped by expert: counts, exclusive prefix offsets [E+1],
+ * and the stable order (expert, token, slot): sorted_to_slot[s] = t*k + j. */
+void oracle_route(const float *logits, int T, int E, int k,
+                  int32_t *topk_ids, float *topk_w, int32_t *counts,
+                  int32_t *offsets, int32_t *sorted_to_slot) {
+    unsigned char *taken = (unsigned char *)malloc((size_t)E);
+    for (int e = 0; e < E; ++e) counts[e] = 0;
+    for (int t = 0; t < T; ++t) {
+        const float *l = logits + (size_t)t * E;
+        memset(taken, 0, (size_t)E);
+        float mx = l[0];
+        for (int e = 1; e < E; ++e) if (l[e] > mx) mx = l[e];
+        float z = 0.0f;
+        for (int e = 0; e < E; ++e) z += expf(l[e] - mx);
+        for (int j = 0; j < k; ++j) {
+            int best = -1;
+            for (int e = 0; e < E; ++e)
+                if (!taken[e] && (best < 0 || l[e] > l[best])) best = e;
+            taken[best] = 1;
+            topk_ids[(size_t)t * k + j] = best;
+            topk_w[(size_t)t * k + j] = expf(l[best] - mx) / z;
+            counts[best] += 1;
+        }
+    }
+    offsets[0] = 0;
+    for (int e = 0; e < E; ++e) offsets[e + 1] = offsets[e] + counts[e];
+    int32_t *fill = (int32_t *)malloc(sizeof(int32_t) * (size_t)E);
+    for (int e = 0; e < E; ++e) fill[e] = offsets[e];
+    for (int t = 0; t < T; ++t)
+        for (int j = 0; j < k; ++j) {
+            int e = topk_ids[(size_t)t * k + j];
+            sorted_to_slot[fill[e]++] = t * k + j;
+        }
+    free(fill);
+    free(taken);
+}
+
+/* -------------------------------------------------------- grouped GEMM
+ * Y_e = X_e W_e^T per expert over that expert's rows (paper, Sec. 3.4), with
+ * both operands NVFP4: the exact sum of dequantised products (binary64;
+ * every product of two code*scale values is exact), times
+ * alpha_e = 1 / (gamma_w[e] * gamma_a[e]) (binary32), rounded once to bf16
+ * (the epilogue factor that folds both tensor scales, Sec. 3.4 / App. D.1).
+ * Rows are the compact expert-sorted rows: expert e owns rows
+ * [offsets[e], offsets[e+1]).  a_codes [R][K/2], a_scales [R][K/32].
+ * Outputs y_bf16 [R][M] and, when abs_sum is not NULL, the tolerance basis
+ * |alpha_e| * sum_k |a_k w_k| per element. */
+void oracle_grouped_gemm(const uint8_t *values, const uint8_t *mask, const uint8_t *scales,
+                         const float *gamma_w, int E, int M, int K,
+                         const uint8_t *a_codes, const uint8_t *a_scales,
+                         const int32_t *offsets, const float *gamma_a,
+                         uint16_t *y_bf16, double *y_exact, double *abs_sum) {
+    double *wq = (double *)malloc(sizeof(double) * (size_t)M * K);   /* code*scale, no gamma */
+    double *aq = (double *)malloc(sizeof(double) * (size_t)K);
+    for (int e = 0; e < E; ++e) {
+        int r0 = offsets[e], r1 = offsets[e + 1];
+        if (r1 <= r0) continue;
+        const uint8_t *ve = values + (size_t)e * M * (K / 4);
+        const uint8_t *me = mask + (size_t)e * M * (K / 16);
+        const uint8_t *se = scales + (size_t)e * M * (K / 32);
+        oracle_unpack_weights(ve, me, se, 1.0f, M, K, wq);
+        volatile float prod = gamma_w[e] * gamma_a[e];
+        float alpha = 1.0f / prod;
+        for (int r = r0; r < r1; ++r) {
+            for (int k = 0; k < K; ++k) {
+                int byte = a_codes[(size_t)r * (K / 2) + k / 2];
+                int c = (k & 1) ? (byte >> 4) : (byte & 15);
+                aq[k] = oracle_e2m1_value(c) * oracle_ue4m3_value(a_scales[(size_t)r * (K / 32) + k / 32]);
+            }
+            for (int m = 0; m < M; ++m) {
+                const double *wr = wq + (size_t)m * K;
+                double s = 0.0, sa = 0.0;
+                for (int k = 0; k < K; ++k) {
+                    double p = aq[k] * wr[k];
+                    s += p;
+                    sa += fabs(p);
+                }
+                double y = (double)alpha * s;
+                y_bf16[(size_t)r * M + m] = double_to_bf16(y);
+                if (y_exact) y_exact[(size_t)r * M + m] = y;
+                if (abs_sum) abs_sum[(size_t)r * M + m] = fabs((double)alpha) * sa;
+            }
+        }
+    }
+    free(aq);
+    free(wq);
+}
+
+/* ----------------------------------------------------------------- SwiGLU
+ * h = SiLU(gate) * up on the bf16 gate_up output: gate = columns [0, I),
+ * up = columns [I, 2I) (paper, App. D.1: SwiGLU output preparation).
+ * SiLU(g) = g / (1 + exp(-g)).  h is rounded once to binary32. */
+void oracle_swiglu(const uint16_t *y_gu, int rows, int I, float *h) {
+    for (int r = 0; r < rows; ++r)
+        for (int i = 0; i < I; ++i) {
+            double g = bf16_to_float(y_gu[(size_t)r * 2 * I + i]);
+            double u = bf16_to_float(y_gu[(size_t)r * 2 * I + I + i]);
+            h[(size_t)r * I + i] = (float)(g / (1.0 + exp(-g)) * u);
+        }
+}
+
+/* ---------------------------------------------------------------- combine
+ * out[t] = sum_{j<k} topk_w[t][j] * Y_down[row of slot (t,j)], binary64,
+ * rounded once to bf16 (router-weighted token combination). */
+void oracle_combine(const uint16_t *y_dn, int H, const float *topk_w,
+                    const int32_t *slot_to_sorted, int T, int k, uint16_t *out) {
+    for (int t = 0; t < T; ++t)
+        for (int h = 0; h < H; ++h) {
+            double s = 0.0;
+            for (int j = 0; j < k; ++j) {
+                int r = slot_to_sorted[(size_t)t * k + j];
+                s += (double)topk_w[(size_t)t * k + j] * bf16_to_float(y_dn[(size_t)r * H + h]);
+            }
+            out[(size_t)t * H + h] = double_to_bf16(s);
+        }
+}
