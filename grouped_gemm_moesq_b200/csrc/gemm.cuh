@@ -1,0 +1,321 @@
+// Grouped sparse NVFP4 GEMM on the sm_100a sparse tensor cores.
+//
+// For every expert e and valid row r of e:
+//   y[r][m] = bf16( alpha_e * sum_k deq(a[r][k]) deq(W_e[m][k]) ),
+//   alpha_e = 1 / (gamma_w[e] gamma_a[e]),
+// in the paper's swap-AB form Y_e^T = W_e X_e^T (Sec. 3.4): the paired-4:8
+// weight is the sparse operand A (M = 128 rows per tile), the token rows of
+// the expert are operand B (N <= TN per tile), both block scales are applied
+// inside the MMA and alpha_e in the epilogue (App. D.1).
+//
+// Design (one CTA per SM, persistent, warp-specialised):
+//   warp 0  TMA producer: per 256-wide K step it loads the compressed weight
+//           tile (128 x 64 B, 64-byte swizzle), the 128-row metadata block
+//           (2 KB) and the weight scales (1 KB) of the kernel form, the token
+//           codes (TN x 128 B, 128-byte swizzle) and their scales (1 KB) into
+//           an S-stage shared-memory ring.
+//   warp 1  MMA issuer (one thread): tcgen05.cp moves metadata and both scale
+//           blocks from shared memory into tensor memory, then two
+//           tcgen05.mma.sp.kind::mxf4nvf4.block_scale (K = 128 dense each)
+//           accumulate in TMEM; tcgen05.commit frees the stage.  Accumulators
+//           are double-buffered in TMEM so the epilogue of tile i overlaps
+//           the main loop of tile i+1.
+//   warps 2-5 epilogue: tcgen05.ld of the fp32 accumulator, times alpha_e,
+//           rounded to bf16 and stored for the valid rows only.
+// Work units are (expert, 128-row weight block, TN-row token block); the
+// per-expert token counts stay on the device and every CTA derives the unit
+// list from them (no host synchronisation).  Units are taken round-robin;
+// consecutive units share the token block, so concurrently running CTAs
+// reuse it from L2 while each streams its own weight block from HBM.
+#pragma once
+#include <cuda.h>
+#include "common.cuh"
+
+namespace moesq {
+
+constexpr int kGemmMaxE = 512;
+constexpr int kGemmThreads = 192;
+
+template <int TN>
+struct GemmCfg {
+  static constexpr int kStages = (TN == 128) ? 6 : 12;
+  static constexpr int kABytes = 128 * 64;       // compressed weight tile, 256 dense K
+  static constexpr int kBBytes = TN * 128;       // token codes, 256 K
+  static constexpr int kEBytes = 128 * 16;       // metadata
+  static constexpr int kSfBytes = 1024;          // 2 x (32 x 16 B)
+  static constexpr int kOffA = 0;
+  static constexpr int kOffB = kOffA + kStages * kABytes;
+  static constexpr int kOffE = kOffB + kStages * kBBytes;
+  static constexpr int kOffSfa = kOffE + kStages * kEBytes;
+  static constexpr int kOffSfb = kOffSfa + kStages * kSfBytes;
+  static constexpr int kOffBar = kOffSfb + kStages * kSfBytes;
+  static constexpr int kNumBars = 2 * kStages + 5;  // full, empty, acc_full[2], acc_empty[2], drain
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kOffTab = kOffMisc + 16;
+  static constexpr int kSmemBytes = kOffTab + (3 * kGemmMaxE + 1) * 4 + 1024;
+  static constexpr uint32_t kTmemCols = (TN == 128) ? 512 : 128;
+  static constexpr uint32_t kColE = 2 * TN;
+  static constexpr uint32_t kColSfa = 2 * TN + 4;
+  static constexpr uint32_t kColSfb = 2 * TN + 12;
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+  static_assert(kColSfb + 8 <= kTmemCols, "tensor memory");
+};
+
+struct GemmParams {
+  const uint8_t* kmeta;
+  const uint8_t* kscales;
+  const uint8_t* a_scales;
+  const float* gamma_w;
+  const float* gamma_a;
+  const int32_t* counts;
+  const int32_t* row_offsets;
+  uint16_t* y;
+  int E, M, K, rows_cap;
+  uint64_t timeout_ns;
+};
+
+struct Tile {
+  int e, mb, row0, nvalid, nmma, q;
+};
+
+// Unit t -> (expert, weight block, token block).  ntp = per-expert prefix of
+// token blocks, rstart = aligned row start, cnt = rows of the expert.
+template <int TN>
+__device__ __forceinline__ Tile decode_tile(int t, int MB, int E, const int* ntp, const int* rstart, const int* cnt) {
+  Tile tl;
+  const int g = t / MB;
+  tl.mb = t - g * MB;
+  int lo = 0, hi = E - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (ntp[mid] <= g) lo = mid; else hi = mid - 1;
+  }
+  tl.e = lo;
+  const int nb = g - ntp[lo];
+  tl.row0 = rstart[lo] + nb * TN;
+  tl.nvalid = min(TN, cnt[lo] - nb * TN);
+  tl.nmma = (tl.nvalid + 15) & ~15;
+  tl.q = (tl.row0 & 127) >> 5;
+  return tl;
+}
+
+template <int TN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                           const GemmParams p) {
+  using C = GemmCfg<TN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int MB = p.M / 128, KT = p.K / 256, KB = p.K / 128, E = p.E;
+
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  int* ntp = reinterpret_cast<int*>(smem + C::kOffTab);   // [E+1]
+  int* rstart = ntp + kGemmMaxE + 1;                       // [E]
+  int* cnt = rstart + kGemmMaxE;                           // [E]
+  auto bar = [&](int i) { return sbase + C::kOffBar + 8u * (uint32_t)i; };
+  auto full_bar = [&](int s) { return bar(s); };
+  auto empty_bar = [&](int s) { return bar(C::kStages + s); };
+  auto accf_bar = [&](int b) { return bar(2 * C::kStages + b); };
+  auto acce_bar = [&](int b) { return bar(2 * C::kStages + 2 + b); };
+  const uint32_t drain_bar = bar(2 * C::kStages + 4);
+
+  // ---------------------------------------------------------------- set-up
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(accf_bar(b), 1); mbar_init(acce_bar(b), 4); }
+    mbar_init(drain_bar, 1);
+    fence_barrier_init();
+    misc[1] = 0;
+    prefetch_tmap(&tm_a);
+    prefetch_tmap(&tm_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(misc), C::kTmemCols);
+    tmem_relinquish();
+  }
+  // expert table; validate the routing counts against the aligned row space
+  int local_bad = 0;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int c = p.counts[e], r0 = p.row_offsets[e], r1 = p.row_offsets[e + 1];
+    const bool ok = c >= 0 && r0 >= 0 && (r0 & 127) == 0 && r1 - r0 == ((c + 127) & ~127) && r1 <= p.rows_cap;
+    local_bad |= ok ? 0 : 1;
+    cnt[e] = ok ? c : 0;
+    rstart[e] = r0;
+    ntp[e + 1] = ok ? (c + TN - 1) / TN : 0;
+  }
+  tc_fence_before();
+  const int bad = __syncthreads_or(local_bad);
+  tc_fence_after();
+  if (warp == 0) {                      // exclusive prefix of token blocks, in place
+    const int per = (E + 31) / 32, e0 = lane * per;   // per <= 16 (E <= 512)
+    int vals[16];
+    int sum = 0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      vals[i] = (i < per && e0 + i < E) ? ntp[e0 + i + 1] : 0;
+      sum += vals[i];
+    }
+    int inc = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += v;
+    }
+    __syncwarp();                       // every lane has read before any lane writes
+    int run = inc - sum;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      if (i < per && e0 + i < E) { ntp[e0 + i] = run; run += vals[i]; }
+    }
+    if (lane == 31) ntp[E] = inc;
+    if (lane == 0 && bad && blockIdx.x == 0) record_error(kWhereGemmCounts, kErrFault);
+  }
+  __syncthreads();
+  const uint32_t tmem = misc[0];
+  const int total = bad ? 0 : ntp[E] * MB;
+
+  // ---------------------------------------------------------------- roles
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_x = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0, issued_parity = 0;     // per-stage bits for the drain on abort
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const Tile tl = decode_tile<TN>(t, MB, E, ntp, rstart, cnt);
+        const int nbox = (tl.nmma + 31) >> 5;
+        const uint32_t bytes = C::kABytes + C::kEBytes + 2 * C::kSfBytes + nbox * 4096;
+        const int64_t wblk = (int64_t)tl.e * MB + tl.mb;
+        const uint8_t* meta = p.kmeta + wblk * KT * 2048;
+        const uint8_t* wsc = p.kscales + wblk * KB * 512;
+        const uint8_t* xsc = p.a_scales + (int64_t)(tl.row0 >> 7) * KB * 512;
+        const int wrow = tl.e * p.M + tl.mb * 128;
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, p.timeout_ns, abort_flag)) {
+            record_error(kWhereGemmProducer, kErrTimeout);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          const uint32_t fb = full_bar(stage);
+          mbar_arrive_expect_tx(fb, bytes);
+          tma_load_2d(sbase + C::kOffA + stage * C::kABytes, &tm_a, fb, kt * 64, wrow, pol_w);
+          bulk_load(sbase + C::kOffE + stage * C::kEBytes, meta + kt * 2048, 2048, fb, pol_w);
+          bulk_load(sbase + C::kOffSfa + stage * C::kSfBytes, wsc + kt * 1024, 1024, fb, pol_w);
+          bulk_load(sbase + C::kOffSfb + stage * C::kSfBytes, xsc + kt * 1024, 1024, fb, pol_x);
+          for (int i = 0; i < nbox; ++i)
+            tma_load_2d(sbase + C::kOffB + stage * C::kBBytes + i * 4096, &tm_b, fb, kt * 128, tl.row0 + 32 * i,
+                        pol_x);
+          issued |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {                        // let the copies in flight land before the CTA exits
+        int zero = 0;
+        for (int s = 0; s < C::kStages; ++s)
+          if (issued >> s & 1u) mbar_wait(full_bar(s), (issued_parity >> s) & 1u, p.timeout_ns, &zero);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true, any = false;
+      int it = 0;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
+        const Tile tl = decode_tile<TN>(t, MB, E, ntp, rstart, cnt);
+        const int buf = it & 1;
+        const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+        if (!mbar_wait(acce_bar(buf), aph ^ 1u, p.timeout_ns, abort_flag)) {
+          record_error(kWhereGemmMma, kErrTimeout);
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(buf * TN);
+        const uint32_t idesc = idesc_sp_nvf4((uint32_t)tl.nmma);
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!mbar_wait(full_bar(stage), phase, p.timeout_ns, abort_flag)) {
+            record_error(kWhereGemmMma, kErrTimeout);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = sbase + C::kOffA + stage * C::kABytes;
+          const uint32_t sb = sbase + C::kOffB + stage * C::kBBytes;
+          const uint32_t se = sbase + C::kOffE + stage * C::kEBytes;
+          const uint32_t ssa = sbase + C::kOffSfa + stage * C::kSfBytes;
+          const uint32_t ssb = sbase + C::kOffSfb + stage * C::kSfBytes;
+          tc_cp_128x128b(tmem + C::kColE, smem_desc(se, 16, 128, 0));
+          tc_cp_32x128b_x4(tmem + C::kColSfa, smem_desc(ssa, 16, 128, 0));
+          tc_cp_32x128b_x4(tmem + C::kColSfa + 4, smem_desc(ssa + 512, 16, 128, 0));
+          tc_cp_32x128b_x4(tmem + C::kColSfb, smem_desc(ssb, 16, 128, 0));
+          tc_cp_32x128b_x4(tmem + C::kColSfb + 4, smem_desc(ssb + 512, 16, 128, 0));
+#pragma unroll
+          for (int kb = 0; kb < 2; ++kb) {
+            const uint64_t adesc = smem_desc(sa + kb * 32, 16, 512, 4);     // 64-byte swizzle
+            const uint64_t bdesc = smem_desc(sb + kb * 64, 16, 1024, 2);    // 128-byte swizzle
+            tc_mma_sp_nvf4(d_tmem, adesc, bdesc, tmem + C::kColE + 2 * kb, idesc, tmem + C::kColSfa + 4 * kb,
+                           tmem + C::kColSfb + 4 * kb + tl.q, (kt | kb) != 0 ? 1u : 0u);
+          }
+          any = true;
+          tc_commit(empty_bar(stage));
+          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+        }
+        if (ok) tc_commit(accf_bar(buf));
+      }
+      if (!ok && any) {                 // drain the MMAs in flight before TMEM is released
+        int zero = 0;
+        tc_commit(drain_bar);
+        mbar_wait(drain_bar, 0, p.timeout_ns, &zero);
+      }
+    }
+  } else {
+    const int quad = warp & 3;          // TMEM lanes 32*quad .. 32*quad+31
+    int it = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+      const Tile tl = decode_tile<TN>(t, MB, E, ntp, rstart, cnt);
+      const int buf = it & 1;
+      const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+      if (!mbar_wait(accf_bar(buf), aph, p.timeout_ns, abort_flag)) {
+        if (lane == 0) { record_error(kWhereGemmEpilogue, kErrTimeout); *abort_flag = 1; }
+        break;
+      }
+      tc_fence_after();
+      const float alpha = __frcp_rn(__fmul_rn(p.gamma_w[tl.e], p.gamma_a[tl.e]));
+      const int m = tl.mb * 128 + quad * 32 + lane;
+      const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * TN);
+      uint16_t* yrow = p.y + (int64_t)tl.row0 * p.M + m;
+      for (int c0 = 0; c0 < tl.nmma; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(taddr + c0, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int n = c0 + j;
+          if (n < tl.nvalid)
+            yrow[(int64_t)n * p.M] = (uint16_t)f32_to_bf16_bits(__fmul_rn(alpha, __uint_as_float(r[j])));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acce_bar(buf));
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace moesq

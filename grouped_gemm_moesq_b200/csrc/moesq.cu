@@ -1,0 +1,506 @@
+// moesq C ABI (include/moesq.h): argument checks, launch configuration,
+// tensor-map construction and the MoE layer composition.  Single
+// translation unit so the device error word is shared by every kernel.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/moesq.h"
+#include "common.cuh"
+#include "gemm.cuh"
+#include "pack.cuh"
+#include "quant.cuh"
+#include "route.cuh"
+
+using namespace moesq;
+
+namespace {
+
+uint64_t g_timeout_ns = 2000000000ull;
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+#define MOESQ_CUDA(call)                                   \
+  do {                                                     \
+    cudaError_t err_ = (call);                             \
+    if (err_ != cudaSuccess) return MOESQ_ERR_CUDA;        \
+  } while (0)
+
+#define MOESQ_TRY(call)                                    \
+  do {                                                     \
+    moesq_status st_ = (call);                             \
+    if (st_ != MOESQ_OK) return st_;                       \
+  } while (0)
+
+inline moesq_status last_launch() {
+  return cudaGetLastError() == cudaSuccess ? MOESQ_OK : MOESQ_ERR_CUDA;
+}
+
+struct DeviceInfo {
+  int sms = 0;
+  bool gemm_attr32 = false, gemm_attr128 = false;
+};
+
+DeviceInfo& device_info() {
+  static DeviceInfo info[64];
+  static std::mutex mu;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(mu);
+  DeviceInfo& d = info[dev & 63];
+  if (d.sms == 0) cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+  return d;
+}
+
+inline int grid_for(int64_t work_items, int per_block, int sms) {
+  const int64_t want = (work_items + per_block - 1) / per_block;
+  return (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)sms * 32));
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D uint8 tensor map: rows x row_bytes, box of box_rows x box_bytes.
+bool make_tmap(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows, uint32_t box_bytes,
+               uint32_t box_rows, CUtensorMapSwizzle swz) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {row_bytes, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_bytes, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+moesq_status check_weights(const moesq_weights* w) {
+  if (!w) return MOESQ_ERR_INVALID_ARG;
+  if (w->E < 1 || w->E > kGemmMaxE || w->M < 128 || w->K < 256) return MOESQ_ERR_UNSUPPORTED_SHAPE;
+  if (w->M % 128 || w->K % 256) return MOESQ_ERR_UNSUPPORTED_SHAPE;
+  if (!w->values || !w->mask || !w->scales || !w->global_scale || !w->kmeta || !w->kscales)
+    return MOESQ_ERR_INVALID_ARG;
+  if (!aligned(w->values, 16) || !aligned(w->kmeta, 16) || !aligned(w->kscales, 16) || !aligned(w->mask, 2) ||
+      !aligned(w->global_scale, 4))
+    return MOESQ_ERR_INVALID_ARG;
+  if ((int64_t)w->E * w->M >= (int64_t)1 << 31) return MOESQ_ERR_UNSUPPORTED_SHAPE;
+  return MOESQ_OK;
+}
+
+moesq_status check_routing(const moesq_routing* rt) {
+  if (!rt) return MOESQ_ERR_INVALID_ARG;
+  if (rt->T < 1 || rt->E < 1 || rt->E > kRouteMaxE || rt->k < 1 || rt->k > std::min(rt->E, 32))
+    return MOESQ_ERR_UNSUPPORTED_SHAPE;
+  if (!rt->topk_ids || !rt->topk_w || !rt->counts || !rt->offsets || !rt->row_offsets || !rt->sorted_to_slot ||
+      !rt->slot_to_row)
+    return MOESQ_ERR_INVALID_ARG;
+  if (rt->rows_cap % 128 || rt->rows_cap < moesq_rows_capacity(rt->T, rt->k, rt->E)) return MOESQ_ERR_INVALID_ARG;
+  return MOESQ_OK;
+}
+
+template <int TN>
+moesq_status launch_gemm(const moesq_weights* w, const uint8_t* a_codes, const uint8_t* a_scales, int rows_cap,
+                         const int32_t* counts, const int32_t* row_offsets, const float* gamma_a, uint16_t* y,
+                         int num_ctas, cudaStream_t s) {
+  using C = GemmCfg<TN>;
+  DeviceInfo& di = device_info();
+  bool& attr = (TN == 128) ? di.gemm_attr128 : di.gemm_attr32;
+  if (!attr) {
+    MOESQ_CUDA(cudaFuncSetAttribute(grouped_sparse_gemm_kernel<TN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    C::kSmemBytes));
+    attr = true;
+  }
+  CUtensorMap tma, tmb;
+  if (!make_tmap(&tma, w->values, (uint64_t)w->K / 4, (uint64_t)w->E * w->M, 64, 128,
+                 CU_TENSOR_MAP_SWIZZLE_64B))
+    return MOESQ_ERR_CUDA;
+  if (!make_tmap(&tmb, a_codes, (uint64_t)w->K / 2, (uint64_t)rows_cap, 128, 32, CU_TENSOR_MAP_SWIZZLE_128B))
+    return MOESQ_ERR_CUDA;
+  GemmParams p;
+  p.kmeta = w->kmeta;
+  p.kscales = w->kscales;
+  p.a_scales = a_scales;
+  p.gamma_w = w->global_scale;
+  p.gamma_a = gamma_a;
+  p.counts = counts;
+  p.row_offsets = row_offsets;
+  p.y = y;
+  p.E = w->E;
+  p.M = w->M;
+  p.K = w->K;
+  p.rows_cap = rows_cap;
+  p.timeout_ns = g_timeout_ns;
+  const int grid = num_ctas > 0 ? num_ctas : di.sms;
+  grouped_sparse_gemm_kernel<TN><<<grid, kGemmThreads, C::kSmemBytes, s>>>(tma, tmb, p);
+  return last_launch();
+}
+
+// Layer workspace carve-up.
+struct LayerWs {
+  int32_t *topk_ids, *counts, *offsets, *row_offsets, *sorted_to_slot, *slot_to_row, *route_ws;
+  float* topk_w;
+  uint8_t *a_codes, *a_scales, *h_codes, *h_scales;
+  uint16_t *y_gu, *y_dn;
+  uint16_t* x_in;    // host variant only
+  float* logits_in;  // host variant only
+  uint16_t* out;     // host variant only
+  int rows_cap;
+  size_t bytes;
+};
+
+LayerWs carve(void* base, int T, int k, int E, int H, int I, bool host_io) {
+  LayerWs w;
+  std::memset(&w, 0, sizeof(w));
+  const int64_t R = (int64_t)T * k;
+  const int64_t rc = moesq_rows_capacity(T, k, E);
+  w.rows_cap = (int)rc;
+  uint8_t* p = static_cast<uint8_t*>(base);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    uint8_t* q = p ? p + off : nullptr;
+    off += align256(bytes);
+    return q;
+  };
+  w.topk_ids = reinterpret_cast<int32_t*>(take(R * 4));
+  w.topk_w = reinterpret_cast<float*>(take(R * 4));
+  w.counts = reinterpret_cast<int32_t*>(take((size_t)E * 4));
+  w.offsets = reinterpret_cast<int32_t*>(take((size_t)(E + 1) * 4));
+  w.row_offsets = reinterpret_cast<int32_t*>(take((size_t)(E + 1) * 4));
+  w.sorted_to_slot = reinterpret_cast<int32_t*>(take(R * 4));
+  w.slot_to_row = reinterpret_cast<int32_t*>(take(R * 4));
+  w.route_ws = reinterpret_cast<int32_t*>(take(moesq_route_workspace_bytes(T, E)));
+  w.a_codes = take((size_t)rc * H / 2);
+  w.a_scales = take((size_t)rc * H / 32);
+  w.y_gu = reinterpret_cast<uint16_t*>(take((size_t)rc * 2 * I * 2));
+  w.h_codes = take((size_t)rc * I / 2);
+  w.h_scales = take((size_t)rc * I / 32);
+  w.y_dn = reinterpret_cast<uint16_t*>(take((size_t)rc * H * 2));
+  if (host_io) {
+    w.x_in = reinterpret_cast<uint16_t*>(take((size_t)T * H * 2));
+    w.logits_in = reinterpret_cast<float*>(take((size_t)T * E * 4));
+    w.out = reinterpret_cast<uint16_t*>(take((size_t)T * H * 2));
+  }
+  w.bytes = off;
+  return w;
+}
+
+moesq_routing routing_of(const LayerWs& w, int T, int E, int k) {
+  moesq_routing rt;
+  rt.T = T;
+  rt.E = E;
+  rt.k = k;
+  rt.rows_cap = w.rows_cap;
+  rt.topk_ids = w.topk_ids;
+  rt.topk_w = w.topk_w;
+  rt.counts = w.counts;
+  rt.offsets = w.offsets;
+  rt.row_offsets = w.row_offsets;
+  rt.sorted_to_slot = w.sorted_to_slot;
+  rt.slot_to_row = w.slot_to_row;
+  return rt;
+}
+
+moesq_status check_layer(int T, int k, const moesq_weights* w_gu, const moesq_weights* w_dn) {
+  MOESQ_TRY(check_weights(w_gu));
+  MOESQ_TRY(check_weights(w_dn));
+  if (T < 1 || k < 1) return MOESQ_ERR_INVALID_ARG;
+  if (w_gu->E != w_dn->E) return MOESQ_ERR_INVALID_ARG;
+  const int H = w_gu->K, I2 = w_gu->M;
+  if (I2 % 2 || w_dn->K != I2 / 2 || w_dn->M != H) return MOESQ_ERR_INVALID_ARG;
+  if (k > std::min(w_gu->E, 32)) return MOESQ_ERR_UNSUPPORTED_SHAPE;
+  if ((I2 / 2) % 256) return MOESQ_ERR_UNSUPPORTED_SHAPE;
+  return MOESQ_OK;
+}
+
+moesq_status layer_body(const uint16_t* x, const float* logits, int T, int k, const moesq_weights* w_gu,
+                        const moesq_weights* w_dn, const float* ga_gu, const float* ga_dn, uint16_t* out,
+                        const LayerWs& ws, cudaStream_t s) {
+  const int E = w_gu->E, H = w_gu->K, I = w_gu->M / 2;
+  moesq_routing rt = routing_of(ws, T, E, k);
+  MOESQ_TRY(moesq_route_permute(logits, &rt, ws.route_ws, moesq_route_workspace_bytes(T, E), s));
+  MOESQ_TRY(moesq_quantize_act(x, T, H, &rt, ga_gu, rt.rows_cap, ws.a_codes, ws.a_scales, s));
+  MOESQ_TRY(moesq_grouped_sparse_gemm(w_gu, ws.a_codes, ws.a_scales, rt.rows_cap, rt.counts, rt.row_offsets, ga_gu,
+                                      ws.y_gu, nullptr, s));
+  MOESQ_TRY(moesq_swiglu_quant(ws.y_gu, I, &rt, ga_dn, ws.h_codes, ws.h_scales, s));
+  MOESQ_TRY(moesq_grouped_sparse_gemm(w_dn, ws.h_codes, ws.h_scales, rt.rows_cap, rt.counts, rt.row_offsets, ga_dn,
+                                      ws.y_dn, nullptr, s));
+  MOESQ_TRY(moesq_combine(ws.y_dn, H, &rt, out, s));
+  return MOESQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moesq_status_str(moesq_status s) {
+  switch (s) {
+    case MOESQ_OK: return "ok";
+    case MOESQ_ERR_INVALID_ARG: return "invalid argument";
+    case MOESQ_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case MOESQ_ERR_CUDA: return "CUDA error";
+    case MOESQ_ERR_TIMEOUT: return "device wait timed out";
+    case MOESQ_ERR_DEVICE_FAULT: return "device-side validation failed";
+    case MOESQ_ERR_WORKSPACE: return "workspace too small";
+  }
+  return "unknown status";
+}
+
+const char* moesq_version(void) { return "moesq 0.1 sm_100a"; }
+
+moesq_status moesq_get_device_error(void* stream, int32_t* device_code) {
+  cudaStream_t s = as_stream(stream);
+  MOESQ_CUDA(cudaStreamSynchronize(s));
+  int v = 0, zero = 0;
+  MOESQ_CUDA(cudaMemcpyFromSymbol(&v, g_error_word, sizeof(int)));
+  MOESQ_CUDA(cudaMemcpyToSymbol(g_error_word, &zero, sizeof(int)));
+  if (device_code) *device_code = v;
+  if (v == 0) return MOESQ_OK;
+  return (v & 0xFF) == kErrTimeout ? MOESQ_ERR_TIMEOUT : MOESQ_ERR_DEVICE_FAULT;
+}
+
+void moesq_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns = ns ? ns : 1; }
+
+size_t moesq_weights_bytes(int E, int M, int K, size_t* per_tensor) {
+  const size_t emk = (size_t)E * M * K;
+  size_t t[6] = {emk / 4, emk / 16, emk / 32, (size_t)E * 4, emk / 16, emk / 32};
+  size_t sum = 0;
+  for (int i = 0; i < 6; ++i) {
+    if (per_tensor) per_tensor[i] = t[i];
+    sum += align256(t[i]);
+  }
+  return sum;
+}
+
+moesq_status moesq_pack_weights(const uint16_t* w_bf16, int e_begin, int e_count, const moesq_weights* out,
+                                void* stream) {
+  MOESQ_TRY(check_weights(out));
+  if (!w_bf16 || !aligned(w_bf16, 16)) return MOESQ_ERR_INVALID_ARG;
+  if (e_begin < 0 || e_count < 1 || e_begin + e_count > out->E) return MOESQ_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  const int sms = device_info().sms;
+  const int M = out->M, K = out->K;
+  float* gamma = out->global_scale + e_begin;
+  MOESQ_CUDA(cudaMemsetAsync(gamma, 0, sizeof(float) * e_count, s));
+  const int64_t groups_per_expert = (int64_t)M * K / 8;
+  const int64_t n_groups = groups_per_expert * e_count;
+  pack_amax_kernel<<<grid_for(n_groups, 256, sms), 256, 0, s>>>(w_bf16, n_groups, groups_per_expert,
+                                                                 reinterpret_cast<unsigned int*>(gamma));
+  MOESQ_TRY(last_launch());
+  pack_gamma_kernel<<<(e_count + 255) / 256, 256, 0, s>>>(gamma, e_count);
+  MOESQ_TRY(last_launch());
+  PackOut po{out->values, out->mask, out->scales, out->global_scale, out->kmeta, out->kscales};
+  const int64_t n_blocks = (int64_t)e_count * M * (K / 32);
+  pack_blocks_kernel<<<grid_for(n_blocks, 256, sms), 256, 0, s>>>(w_bf16, e_begin, n_blocks, M, K, po);
+  return last_launch();
+}
+
+int64_t moesq_rows_capacity(int T, int k, int E) {
+  if (T < 0 || k < 0 || E < 0) return 0;
+  const int64_t R = (int64_t)T * k;
+  const int64_t rc = R + 127 * std::min<int64_t>(E, R);
+  return std::max<int64_t>(128, (rc + 127) / 128 * 128);
+}
+
+size_t moesq_route_workspace_bytes(int T, int E) {
+  const size_t nblk = (size_t)(T + kRouteTPB - 1) / kRouteTPB;
+  return align256(nblk * (size_t)E * 4);
+}
+
+moesq_status moesq_route_permute(const float* logits, const moesq_routing* rt, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  MOESQ_TRY(check_routing(rt));
+  if (!logits) return MOESQ_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < moesq_route_workspace_bytes(rt->T, rt->E)) return MOESQ_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  const int nblk = (rt->T + kRouteTPB - 1) / kRouteTPB;
+  int32_t* bc = static_cast<int32_t*>(workspace);
+  const size_t smem = (size_t)rt->E * kRouteWords * 4;
+  route_topk_kernel<<<nblk, 256, smem, s>>>(logits, rt->T, rt->E, rt->k, rt->topk_ids, rt->topk_w, bc);
+  MOESQ_TRY(last_launch());
+  route_scan_kernel<<<1, 1024, 0, s>>>(bc, nblk, rt->E, rt->counts, rt->offsets, rt->row_offsets);
+  MOESQ_TRY(last_launch());
+  route_scatter_kernel<<<nblk, 256, smem, s>>>(rt->T, rt->E, rt->k, rt->topk_ids, bc, rt->offsets, rt->row_offsets,
+                                               rt->sorted_to_slot, rt->slot_to_row);
+  return last_launch();
+}
+
+moesq_status moesq_quantize_act(const uint16_t* x_bf16, int T, int K, const moesq_routing* rt, const float* gamma,
+                                int rows_cap, uint8_t* codes, uint8_t* scales, void* stream) {
+  if (!x_bf16 || !gamma || !codes || !scales) return MOESQ_ERR_INVALID_ARG;
+  if (T < 1 || K < 256 || K % 256) return MOESQ_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(x_bf16, 16) || !aligned(codes, 4)) return MOESQ_ERR_INVALID_ARG;
+  if (rows_cap < 128 || rows_cap % 128) return MOESQ_ERR_INVALID_ARG;
+  int k = 1, E = 1;
+  const int32_t* ids = nullptr;
+  const int32_t* s2r = nullptr;
+  if (rt) {
+    MOESQ_TRY(check_routing(rt));
+    if (rt->T != T || rows_cap != rt->rows_cap) return MOESQ_ERR_INVALID_ARG;
+    k = rt->k;
+    E = rt->E;
+    ids = rt->topk_ids;
+    s2r = rt->slot_to_row;
+  } else if (rows_cap < T) {
+    return MOESQ_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = as_stream(stream);
+  const int64_t tasks = (int64_t)T * (rt ? k : 1) * (K / 256);
+  quantize_act_kernel<<<grid_for(tasks, 8, device_info().sms), 256, 0, s>>>(x_bf16, T, K, k, ids, s2r, E, gamma,
+                                                                            rows_cap, codes, scales);
+  return last_launch();
+}
+
+moesq_status moesq_act_global_scale(const uint16_t* x_bf16, int64_t n, float* gamma_out, void* stream) {
+  if (!x_bf16 || !gamma_out || n < 1) return MOESQ_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  MOESQ_CUDA(cudaMemsetAsync(gamma_out, 0, sizeof(float), s));
+  amax_bf16_kernel<<<grid_for(n, 256 * 8, device_info().sms), 256, 0, s>>>(
+      x_bf16, n, reinterpret_cast<unsigned int*>(gamma_out));
+  MOESQ_TRY(last_launch());
+  amax_to_gamma_kernel<<<1, 32, 0, s>>>(gamma_out, 1, 0);
+  return last_launch();
+}
+
+moesq_status moesq_grouped_sparse_gemm(const moesq_weights* w, const uint8_t* a_codes, const uint8_t* a_scales,
+                                       int rows_cap, const int32_t* counts, const int32_t* row_offsets,
+                                       const float* gamma_a, uint16_t* y_bf16, const moesq_gemm_config* cfg,
+                                       void* stream) {
+  MOESQ_TRY(check_weights(w));
+  if (!a_codes || !a_scales || !counts || !row_offsets || !gamma_a || !y_bf16) return MOESQ_ERR_INVALID_ARG;
+  if (rows_cap < 128 || rows_cap % 128) return MOESQ_ERR_INVALID_ARG;
+  if (!aligned(a_codes, 16) || !aligned(a_scales, 16) || !aligned(y_bf16, 2)) return MOESQ_ERR_INVALID_ARG;
+  int tile_n = cfg ? cfg->tile_n : 0;
+  const int num_ctas = cfg ? cfg->num_ctas : 0;
+  if (tile_n != 0 && tile_n != 32 && tile_n != 128) return MOESQ_ERR_INVALID_ARG;
+  if (num_ctas < 0) return MOESQ_ERR_INVALID_ARG;
+  if (tile_n == 0) {
+    // The counts stay on the device.  The aligned row capacity, less the
+    // padding of at most 127 rows per expert, bounds the mean rows per expert.
+    const int64_t rows_est = std::max<int64_t>(0, (int64_t)rows_cap - 127 * (int64_t)w->E);
+    tile_n = rows_est / w->E > 64 ? 128 : 32;
+  }
+  cudaStream_t s = as_stream(stream);
+  if (tile_n == 32)
+    return launch_gemm<32>(w, a_codes, a_scales, rows_cap, counts, row_offsets, gamma_a, y_bf16, num_ctas, s);
+  return launch_gemm<128>(w, a_codes, a_scales, rows_cap, counts, row_offsets, gamma_a, y_bf16, num_ctas, s);
+}
+
+moesq_status moesq_swiglu_quant(const uint16_t* y_gu, int I, const moesq_routing* rt, const float* gamma_h,
+                                uint8_t* h_codes, uint8_t* h_scales, void* stream) {
+  MOESQ_TRY(check_routing(rt));
+  if (!y_gu || !gamma_h || !h_codes || !h_scales) return MOESQ_ERR_INVALID_ARG;
+  if (I < 256 || I % 256) return MOESQ_ERR_UNSUPPORTED_SHAPE;
+  const int R = rt->T * rt->k;
+  const int64_t tasks = (int64_t)R * (I / 256);
+  swiglu_quant_kernel<<<grid_for(tasks, 8, device_info().sms), 256, 0, as_stream(stream)>>>(
+      y_gu, I, R, rt->E, rt->offsets, rt->row_offsets, gamma_h, h_codes, h_scales, nullptr);
+  return last_launch();
+}
+
+moesq_status moesq_combine(const uint16_t* y, int H, const moesq_routing* rt, uint16_t* out, void* stream) {
+  MOESQ_TRY(check_routing(rt));
+  if (!y || !out || H < 8 || H % 8) return MOESQ_ERR_INVALID_ARG;
+  if (!aligned(y, 16) || !aligned(out, 16)) return MOESQ_ERR_INVALID_ARG;
+  const int64_t tasks = (int64_t)rt->T * ((H + 255) / 256);
+  combine_kernel<<<grid_for(tasks, 8, device_info().sms), 256, 0, as_stream(stream)>>>(
+      y, H, rt->T, rt->k, rt->topk_w, rt->slot_to_row, rt->rows_cap, out);
+  return last_launch();
+}
+
+size_t moesq_layer_workspace_bytes(int T, int k, int E, int H, int I) {
+  return carve(nullptr, T, k, E, H, I, false).bytes;
+}
+
+size_t moesq_layer_host_workspace_bytes(int T, int k, int E, int H, int I) {
+  return carve(nullptr, T, k, E, H, I, true).bytes;
+}
+
+moesq_status moesq_moe_layer(const uint16_t* x_bf16, const float* logits, int T, int k, const moesq_weights* w_gu,
+                             const moesq_weights* w_dn, const float* gamma_a_gu, const float* gamma_a_dn,
+                             uint16_t* out_bf16, void* workspace, size_t workspace_bytes, void* stream) {
+  MOESQ_TRY(check_layer(T, k, w_gu, w_dn));
+  if (!x_bf16 || !logits || !gamma_a_gu || !gamma_a_dn || !out_bf16) return MOESQ_ERR_INVALID_ARG;
+  const int E = w_gu->E, H = w_gu->K, I = w_gu->M / 2;
+  if (!workspace || !aligned(workspace, 256)) return MOESQ_ERR_INVALID_ARG;
+  LayerWs ws = carve(workspace, T, k, E, H, I, false);
+  if (workspace_bytes < ws.bytes) return MOESQ_ERR_WORKSPACE;
+  return layer_body(x_bf16, logits, T, k, w_gu, w_dn, gamma_a_gu, gamma_a_dn, out_bf16, ws, as_stream(stream));
+}
+
+moesq_status moesq_moe_layer_host(const uint16_t* x_bf16_host, const float* logits_host, int T, int k,
+                                  const moesq_weights* w_gu, const moesq_weights* w_dn, const float* gamma_a_gu,
+                                  const float* gamma_a_dn, uint16_t* out_bf16_host, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  MOESQ_TRY(check_layer(T, k, w_gu, w_dn));
+  if (!x_bf16_host || !logits_host || !gamma_a_gu || !gamma_a_dn || !out_bf16_host) return MOESQ_ERR_INVALID_ARG;
+  const int E = w_gu->E, H = w_gu->K, I = w_gu->M / 2;
+  if (!workspace || !aligned(workspace, 256)) return MOESQ_ERR_INVALID_ARG;
+  LayerWs ws = carve(workspace, T, k, E, H, I, true);
+  if (workspace_bytes < ws.bytes) return MOESQ_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  MOESQ_CUDA(cudaMemcpyAsync(ws.x_in, x_bf16_host, (size_t)T * H * 2, cudaMemcpyHostToDevice, s));
+  MOESQ_CUDA(cudaMemcpyAsync(ws.logits_in, logits_host, (size_t)T * E * 4, cudaMemcpyHostToDevice, s));
+  MOESQ_TRY(layer_body(ws.x_in, ws.logits_in, T, k, w_gu, w_dn, gamma_a_gu, gamma_a_dn, ws.out, ws, s));
+  MOESQ_CUDA(cudaMemcpyAsync(out_bf16_host, ws.out, (size_t)T * H * 2, cudaMemcpyDeviceToHost, s));
+  MOESQ_CUDA(cudaStreamSynchronize(s));
+  return MOESQ_OK;
+}
+
+moesq_status moesq_calibrate_layer(const uint16_t* x_bf16, const float* logits, int T, int k,
+                                   const moesq_weights* w_gu, const moesq_weights* w_dn, float* gamma_a_gu,
+                                   float* gamma_a_dn, void* workspace, size_t workspace_bytes, void* stream) {
+  MOESQ_TRY(check_layer(T, k, w_gu, w_dn));
+  if (!x_bf16 || !logits || !gamma_a_gu || !gamma_a_dn) return MOESQ_ERR_INVALID_ARG;
+  const int E = w_gu->E, H = w_gu->K, I = w_gu->M / 2;
+  if (!workspace || !aligned(workspace, 256)) return MOESQ_ERR_INVALID_ARG;
+  LayerWs ws = carve(workspace, T, k, E, H, I, false);
+  if (workspace_bytes < ws.bytes) return MOESQ_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  const int sms = device_info().sms;
+  moesq_routing rt = routing_of(ws, T, E, k);
+  MOESQ_TRY(moesq_route_permute(logits, &rt, ws.route_ws, moesq_route_workspace_bytes(T, E), s));
+  MOESQ_CUDA(cudaMemsetAsync(gamma_a_gu, 0, sizeof(float) * E, s));
+  routed_amax_kernel<<<grid_for((int64_t)T * k, 8, sms), 256, 0, s>>>(x_bf16, T, H, k, rt.topk_ids, E,
+                                                                       reinterpret_cast<unsigned int*>(gamma_a_gu));
+  MOESQ_TRY(last_launch());
+  amax_to_gamma_kernel<<<1, 1024, 0, s>>>(gamma_a_gu, E, 1);
+  MOESQ_TRY(last_launch());
+  MOESQ_TRY(moesq_quantize_act(x_bf16, T, H, &rt, gamma_a_gu, rt.rows_cap, ws.a_codes, ws.a_scales, s));
+  MOESQ_TRY(moesq_grouped_sparse_gemm(w_gu, ws.a_codes, ws.a_scales, rt.rows_cap, rt.counts, rt.row_offsets,
+                                      gamma_a_gu, ws.y_gu, nullptr, s));
+  MOESQ_CUDA(cudaMemsetAsync(gamma_a_dn, 0, sizeof(float) * E, s));
+  const int R = T * k;
+  swiglu_quant_kernel<<<grid_for((int64_t)R * (I / 256), 8, sms), 256, 0, s>>>(
+      ws.y_gu, I, R, E, rt.offsets, rt.row_offsets, nullptr, nullptr, nullptr,
+      reinterpret_cast<unsigned int*>(gamma_a_dn));
+  MOESQ_TRY(last_launch());
+  amax_to_gamma_kernel<<<1, 1024, 0, s>>>(gamma_a_dn, E, 1);
+  return last_launch();
+}
+
+moesq_status moesq_debug_bounded_wait(uint64_t timeout_ns, void* stream) {
+  debug_wait_kernel<<<1, 32, 0, as_stream(stream)>>>(timeout_ns ? timeout_ns : 1);
+  return last_launch();
+}
+
+}  // extern "C"

@@ -1,0 +1,147 @@
+// Weight packing: bf16 expert weights -> paired-4:8 sparse NVFP4.
+//
+// Support: per group of 8 K elements keep the two pairs of largest
+// w0^2 + w1^2 (binary32), an exact tie keeping the lower pair index
+// (paper App. A Eq. 6 pattern set; model card "exactly 2 pairs are kept").
+// Scales: paper Sec. 3.4 Eq. 5 on the masked weights; values: Eq. 3.
+// Outputs the storage form of the model card (values / mask / scales /
+// gamma) and the kernel form read by the grouped GEMM (kmeta / kscales).
+#pragma once
+#include "common.cuh"
+
+namespace moesq {
+
+// Kept-pair bitmask (bit p = pair p) of one group of 8 values.
+__device__ __forceinline__ uint32_t select_pairs(const float (&w)[8]) {
+  float s[4];
+#pragma unroll
+  for (int p = 0; p < 4; ++p) s[p] = __fadd_rn(__fmul_rn(w[2 * p], w[2 * p]), __fmul_rn(w[2 * p + 1], w[2 * p + 1]));
+  uint32_t bits = 0;
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    int beaten = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (q != p && (s[q] > s[p] || (s[q] == s[p] && q < p))) ++beaten;
+    if (beaten < 2) bits |= 1u << p;
+  }
+  return bits;
+}
+
+__device__ __forceinline__ void load_group(const uint16_t* src, float (&w)[8]) {
+  uint4 v = *reinterpret_cast<const uint4*>(src);
+  w[0] = bf16lo(v.x); w[1] = bf16hi(v.x); w[2] = bf16lo(v.y); w[3] = bf16hi(v.y);
+  w[4] = bf16lo(v.z); w[5] = bf16hi(v.z); w[6] = bf16lo(v.w); w[7] = bf16hi(v.w);
+}
+
+// Pass 1: largest kept |w| per expert, accumulated as float bits (>= 0) with
+// atomicMax into amax_bits[e].  One thread per group of 8.
+__global__ void pack_amax_kernel(const uint16_t* __restrict__ w, int64_t n_groups,
+                                 int64_t groups_per_expert, unsigned int* __restrict__ amax_bits) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g - (threadIdx.x & 31) < n_groups;
+       g += stride) {
+    float a = 0.0f;
+    int64_t e = -1;
+    if (g < n_groups) {
+      float v[8];
+      load_group(w + g * 8, v);
+      uint32_t bits = select_pairs(v);
+#pragma unroll
+      for (int p = 0; p < 4; ++p)
+        if (bits >> p & 1u) a = fmaxf(a, fmaxf(fabsf(v[2 * p]), fabsf(v[2 * p + 1])));
+      e = g / groups_per_expert;
+    }
+    // groups_per_expert is a multiple of 32: a warp never spans two experts
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    if ((threadIdx.x & 31) == 0 && e >= 0) atomicMax(amax_bits + e, __float_as_uint(a));
+  }
+}
+
+// amax bits -> gamma (Eq. 5), in place.
+__global__ void pack_gamma_kernel(float* __restrict__ gamma, int n) {
+  int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) gamma[i] = nvfp4_global_scale(gamma[i]);   // gamma[i] holds amax here
+}
+
+struct PackOut {
+  uint8_t* values;    // [E][M][K/4]
+  uint8_t* mask;      // [E][M][K/16]
+  uint8_t* scales;    // [E][M][K/32]
+  const float* gamma; // [E]
+  uint8_t* kmeta;     // [E][M/128][K/256][128][16]
+  uint8_t* kscales;   // [E][M/128][K/128][512]
+};
+
+// Pass 2: one thread per 32-element block (4 groups, 16 kept values).
+__global__ void pack_blocks_kernel(const uint16_t* __restrict__ w, int e_begin, int64_t n_blocks, int M,
+                                   int K, PackOut out) {
+  const int nb_row = K / 32, KT = K / 256, KB = K / 128, MB = M / 128;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < n_blocks; t += stride) {
+    const int b = (int)(t % nb_row);
+    const int64_t row_local = t / nb_row;          // e_local * M + m
+    const int e = e_begin + (int)(row_local / M);
+    const int m = (int)(row_local % M);
+    const int64_t row = (int64_t)e * M + m;        // row of the full stack
+    const uint16_t* src = w + row_local * K + (int64_t)b * 32;
+
+    float kept[16];                                 // kept values of the block, K order
+    uint32_t bits4[4];
+    float amax = 0.0f;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      float v[8];
+      load_group(src + 8 * g, v);
+      uint32_t bits = select_pairs(v);
+      bits4[g] = bits;
+      int slot = 0;
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        if (bits >> p & 1u) {
+          // slot is 0 or 1; written without dynamic register indexing
+          float x0 = v[2 * p], x1 = v[2 * p + 1];
+          if (slot == 0) { kept[4 * g + 0] = x0; kept[4 * g + 1] = x1; }
+          else           { kept[4 * g + 2] = x0; kept[4 * g + 3] = x1; }
+          amax = fmaxf(amax, fmaxf(fabsf(x0), fabsf(x1)));
+          ++slot;
+        }
+      }
+    }
+    const float gamma = out.gamma[e];
+    const uint32_t code = block_scale_code(gamma, amax);
+    const float s_b = block_step(code, gamma);
+    float h0[8], h1[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) { h0[i] = kept[i]; h1[i] = kept[8 + i]; }
+    uint2 vbytes;
+    vbytes.x = quant8(h0, s_b, code == 0);
+    vbytes.y = quant8(h1, s_b, code == 0);
+
+    // storage form
+    *reinterpret_cast<uint2*>(out.values + row * (K / 4) + (int64_t)b * 8) = vbytes;
+    const uint16_t mk = (uint16_t)(bits4[0] | (bits4[1] << 4) | (bits4[2] << 8) | (bits4[3] << 12));
+    *reinterpret_cast<uint16_t*>(out.mask + row * (K / 16) + (int64_t)b * 2) = mk;
+    out.scales[row * nb_row + b] = (uint8_t)code;
+
+    // kernel form: metadata nibble = i0 | i1 << 2 of the two kept pair indices
+    uint32_t meta = 0;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      const uint32_t bits = bits4[g];
+      const uint32_t i0 = __ffs(bits) - 1;
+      const uint32_t i1 = 31 - __clz(bits);
+      meta |= (i0 | (i1 << 2)) << (4 * g);
+    }
+    const int mb = m >> 7, i = m & 127;
+    const int kt = b >> 3;
+    const int64_t mo = ((((int64_t)e * MB + mb) * KT + kt) * 128 + i) * 16 + (b & 7) * 2;
+    *reinterpret_cast<uint16_t*>(out.kmeta + mo) = (uint16_t)meta;
+    const int kb = b >> 2, s = b & 3;
+    const int64_t so = (((int64_t)e * MB + mb) * KB + kb) * 512 + (i & 31) * 16 + (i >> 5) * 4 + s;
+    out.kscales[so] = (uint8_t)code;
+  }
+}
+
+}  // namespace moesq

@@ -283,3 +283,30 @@ def moe_layer(x_bf16, logits, k, pk_gu: Packed, pk_dn: Packed, gamma_a_gu, gamma
         return out, dict(rt=rt, a_codes=a_c, a_scales=a_s, y_gu=y_gu, h=h, h_codes=h_c,
                          h_scales=h_s, y_dn=y_dn)
     return out
+
+
+def calibrate_layer(x_bf16, logits, k, pk_gu: Packed, pk_dn: Packed):
+    """Static activation global scales from a calibration batch (the
+    definition moesq_calibrate_layer implements): per expert, Eq. 5's gamma
+    of the largest |x| over its routed tokens, then of the largest |h| over
+    its SwiGLU rows computed with those gammas; an expert without tokens
+    takes the largest amax over all experts."""
+    E = pk_gu.E
+    rt = route(logits, k)
+    ex = rt.expert_of_sorted()
+    toks = rt.sorted_to_slot // k
+    xf = np.abs((np.asarray(x_bf16, np.uint16).astype(np.uint32) << 16).view(np.float32))
+    amax = np.zeros(E, np.float32)
+    for s in range(toks.size):
+        amax[ex[s]] = max(amax[ex[s]], xf[toks[s]].max())
+    amax[amax == 0] = amax.max()
+    ga = np.array([global_scale(a) for a in amax], np.float32)
+    a_c, a_s = permute_quantize(x_bf16, rt, ga)
+    y_gu, _ = grouped_gemm(pk_gu, a_c, a_s, rt.offsets, ga)
+    h = np.abs(swiglu(y_gu))
+    amax_h = np.zeros(E, np.float32)
+    for s in range(toks.size):
+        amax_h[ex[s]] = max(amax_h[ex[s]], h[s].max())
+    amax_h[amax_h == 0] = amax_h.max()
+    gh = np.array([global_scale(a) for a in amax_h], np.float32)
+    return ga, gh

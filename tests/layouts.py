@@ -1,0 +1,86 @@
+"""Host-side transforms between the storage form and the kernel layouts that
+include/moesq.h defines (test helpers; numpy only).
+
+* kmeta   [E][M/128][K/256][128][16]: byte b of row i holds the metadata of
+          chunks 2b (low nibble) and 2b+1; a chunk nibble is i0 | i1 << 2 of
+          its two kept pair indices.
+* kscales [E][M/128][K/128][32][4][4] and the activation scale layout
+          [R/128][K/128][32][4][4]: scale of row 32a+b (of a 128-row block),
+          sub-block s of a 128-wide K block, at byte b*16 + a*4 + s.
+* aligned row space: expert e owns rows row_offsets[e] + [0, counts[e]).
+"""
+import numpy as np
+
+
+def mask_to_kmeta(mask: np.ndarray) -> np.ndarray:
+    """mask uint8 [E, M, K/16] (pair bitmask) -> kmeta bytes (flat)."""
+    E, M, K16 = mask.shape
+    K = K16 * 16
+    nib = np.stack([mask & 15, mask >> 4], -1).reshape(E, M, K // 8)          # per chunk bitmask
+    i0 = np.zeros_like(nib)
+    i1 = np.zeros_like(nib)
+    for p in range(3, -1, -1):
+        hit = (nib >> p) & 1 == 1
+        i0 = np.where(hit, p, i0)          # ends with the lowest set bit
+    for p in range(4):
+        hit = (nib >> p) & 1 == 1
+        i1 = np.where(hit, p, i1)          # ends with the highest set bit
+    code = (i0 | (i1 << 2)).astype(np.uint8)                                   # [E, M, K/8]
+    byte = (code[..., 0::2] | (code[..., 1::2] << 4)).astype(np.uint8)         # [E, M, K/16]
+    # [E, MB, 128, KT, 16] -> [E, MB, KT, 128, 16]
+    b = byte.reshape(E, M // 128, 128, K // 256, 16).transpose(0, 1, 3, 2, 4)
+    return np.ascontiguousarray(b).reshape(-1)
+
+
+def kmeta_to_mask(kmeta: np.ndarray, E: int, M: int, K: int) -> np.ndarray:
+    b = kmeta.reshape(E, M // 128, K // 256, 128, 16).transpose(0, 1, 3, 2, 4).reshape(E, M, K // 16)
+    code = np.stack([b & 15, b >> 4], -1).reshape(E, M, K // 8)
+    i0, i1 = code & 3, code >> 2
+    nib = ((1 << i0) | (1 << i1)).astype(np.uint8)
+    return (nib[..., 0::2] | (nib[..., 1::2] << 4)).astype(np.uint8)
+
+
+def scales_to_mma(sc: np.ndarray) -> np.ndarray:
+    """Row-major scales [R, K/32] (R multiple of 128) -> MMA scale layout (flat)."""
+    R, S = sc.shape
+    # [R/128, 4(a), 32(b), K/128, 4(s)] -> [R/128, K/128, 32(b), 4(a), 4(s)]
+    t = sc.reshape(R // 128, 4, 32, S // 4, 4).transpose(0, 3, 2, 1, 4)
+    return np.ascontiguousarray(t).reshape(-1)
+
+
+def mma_to_scales(flat: np.ndarray, R: int, K: int) -> np.ndarray:
+    t = flat.reshape(R // 128, K // 128, 32, 4, 4).transpose(0, 3, 2, 1, 4)
+    return np.ascontiguousarray(t).reshape(R, K // 32)
+
+
+def weight_scales_to_kscales(scales: np.ndarray) -> np.ndarray:
+    E, M, S = scales.shape
+    return np.concatenate([scales_to_mma(scales[e]) for e in range(E)])
+
+
+def kscales_to_weight_scales(flat: np.ndarray, E: int, M: int, K: int) -> np.ndarray:
+    per = M * K // 32
+    return np.stack([mma_to_scales(flat[e * per:(e + 1) * per], M, K) for e in range(E)])
+
+
+def aligned_rows(counts: np.ndarray):
+    """row_offsets [E+1] of the expert-aligned row space."""
+    pad = (counts + 127) // 128 * 128
+    return np.concatenate([[0], np.cumsum(pad)]).astype(np.int32)
+
+
+def compact_to_rows(counts: np.ndarray) -> np.ndarray:
+    """row of every compact (expert-sorted) position."""
+    offs = np.concatenate([[0], np.cumsum(counts)])
+    ro = aligned_rows(counts)
+    rows = np.empty(int(offs[-1]), np.int64)
+    for e in range(counts.size):
+        rows[offs[e]:offs[e + 1]] = ro[e] + np.arange(counts[e])
+    return rows
+
+
+def bf16_ulp(y: np.ndarray) -> np.ndarray:
+    """Spacing of bf16 numbers at |y| (for y != 0)."""
+    a = np.abs(np.asarray(y, np.float64))
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    return np.where(a > 0, 2.0 ** (e - 7), 0.0)

@@ -1,0 +1,173 @@
+"""GPU parity of the grouped sparse GEMM against the oracle:
+|y - y_ref| <= 1e-3 * sum_k |a_k w_k| + one bf16 spacing, per element."""
+import numpy as np
+import pytest
+
+import layouts as L
+import oracle as O
+import synthetic as S
+from gpu_cases import (act_rows_from_compact, gemm_tolerance_ok, pack_gpu_from_np, pack_gpu_generated,
+                       packed_from_oracle, to_dev, to_np, weights_np)
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_isolated(m, pk, counts, K, seed, tile_n, ga_scale=1.0):
+    """Oracle weights + oracle-quantised activations, laid out on the host,
+    through the CUDA GEMM; returns (ok, detail)."""
+    torch = pytest.importorskip("torch")
+    E = counts.size
+    R = int(counts.sum())
+    x = S.activations_bf16_np(seed, max(R, 1), K)
+    ga = np.array([np.float32(O.act_global_scale(x)) * np.float32(ga_scale * (1 + e % 3))
+                   for e in range(E)], np.float32)
+    offs = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    ex = np.repeat(np.arange(E), counts)
+    codes = np.zeros((R, K // 2), np.uint8)
+    scales = np.zeros((R, K // 32), np.uint8)
+    for e in range(E):
+        if counts[e]:
+            c, s = O.quantize_rows_bf16(x[offs[e]:offs[e + 1]], ga[e])
+            codes[offs[e]:offs[e + 1]], scales[offs[e]:offs[e + 1]] = c, s
+    y_ref, basis = O.grouped_gemm(pk, codes, scales, offs, ga)
+    pw = packed_from_oracle(m, pk)
+    c_rows, s_mma, rc = act_rows_from_compact(codes, scales, counts, K)
+    M = pk.values.shape[1]
+    y = torch.full((rc, M), float("nan"), dtype=torch.bfloat16, device="cuda")
+    m.moesq_grouped_sparse_gemm(pw, to_dev(c_rows), to_dev(s_mma), rc, to_dev(counts.astype(np.int32)),
+                                to_dev(L.aligned_rows(counts)), to_dev(ga), y, tile_n=tile_n)
+    st, word = m.moesq_get_device_error()
+    assert st == 0, "device error word %#x" % word
+    rows = L.compact_to_rows(counts)
+    yg = to_np(y)[rows]
+    ok, err, bound, bad = gemm_tolerance_ok(yg, y_ref, basis)
+    return ok, (err.max(), np.argwhere(bad)[:5], ex)
+
+
+@pytest.mark.parametrize("tile_n", [32, 128])
+def test_gemm_tiny_config(cuda_lib, tile_n):
+    """E=8, K=512, M=256 with the token counts of 64 tokens routed top-2."""
+    E, M, K, T, k = 8, 256, 512, 64, 2
+    pk = O.pack_weights(weights_np(1, 0, E, M, K))
+    counts = O.route(S.uniform_logits_np(1, T, E), k).counts
+    ok, info = _run_isolated(cuda_lib, pk, counts, K, 2, tile_n)
+    assert ok, info[:2]
+
+
+@pytest.mark.parametrize("tile_n", [32, 128])
+@pytest.mark.parametrize("counts", [
+    [0, 1, 0, 5, 0, 0, 0, 2],              # empty experts, single rows
+    [129, 0, 31, 33, 1, 16, 17, 300],      # ragged: several token blocks, partial last blocks
+    [0, 0, 0, 0, 0, 0, 0, 512],            # all rows on one expert
+    [128, 256, 32, 64, 96, 160, 192, 224], # exact multiples of the token block
+])
+def test_gemm_edge_counts(cuda_lib, tile_n, counts):
+    E, M, K = 8, 256, 512
+    pk = O.pack_weights(weights_np(3, 0, E, M, K))
+    ok, info = _run_isolated(cuda_lib, pk, np.array(counts, np.int64), K, 4, tile_n)
+    assert ok, info[:2]
+
+
+def test_gemm_multi_k_tiles_and_m_blocks(cuda_lib):
+    """K = 2048 (8 K steps, deeper than the smem ring wraps) and M = 1536."""
+    E, M, K = 3, 1536, 2048
+    pk = O.pack_weights(weights_np(5, 0, E, M, K))
+    ok, info = _run_isolated(cuda_lib, pk, np.array([7, 0, 40]), K, 6, 0)
+    assert ok, info[:2]
+
+
+def test_gemm_saturating_activation_scale(cuda_lib):
+    """gamma_a too large: scales clip at 448 and codes at 6; still exact math."""
+    E, M, K = 2, 128, 256
+    pk = O.pack_weights(weights_np(7, 0, E, M, K))
+    ok, info = _run_isolated(cuda_lib, pk, np.array([20, 3]), K, 8, 32, ga_scale=64.0)
+    assert ok, info[:2]
+
+
+def test_gemm_full_path_30b_class(cuda_lib):
+    """30B-class gate_up (E=128, top-8, K=2048, M=1536, T=256): CUDA pack,
+    route, dispatch-quantise and GEMM, checked on the rows of 6 experts."""
+    torch = pytest.importorskip("torch")
+    m = cuda_lib
+    E, M, K, T, k = 128, 1536, 2048, 256, 8
+    pw = pack_gpu_generated(m, 11, 0, E, M, K)
+    x = S.activations_bf16_np(11, T, K)
+    lg = S.uniform_logits_np(11, T, E)
+    rt = O.route(lg, k)
+    ga = np.full(E, O.act_global_scale(x), np.float32)
+    rb = m.RoutingBuffers(T, E, k)
+    m.moesq_route_permute(to_dev(lg), rb)
+    codes, scales = m.act_buffers(rb.rows_cap, K)
+    m.moesq_quantize_act(to_dev(x), T, K, rb, to_dev(ga), rb.rows_cap, codes, scales)
+    y = torch.full((rb.rows_cap, M), float("nan"), dtype=torch.bfloat16, device="cuda")
+    m.moesq_grouped_sparse_gemm(pw, codes, scales, rb.rows_cap, rb.counts, rb.row_offsets, to_dev(ga), y)
+    assert m.moesq_get_device_error()[0] == 0
+    yg_all = to_np(y)
+    ro = L.aligned_rows(rt.counts)
+    for e in (0, 17, 64, 101, 126, 127):
+        n = int(rt.counts[e])
+        if n == 0:
+            continue
+        pk = O.pack_weights(S.expert_weights_bf16_np(11, 0, e, M, K)[None])
+        s0 = rt.offsets[e]
+        toks = rt.sorted_to_slot[s0:s0 + n] // k
+        c, s = O.quantize_rows_bf16(x[toks], ga[e])
+        y_ref, basis = O.grouped_gemm(pk, c, s, np.array([0, n], np.int32), ga[e:e + 1])
+        ok, err, bound, bad = gemm_tolerance_ok(yg_all[ro[e]:ro[e] + n], y_ref, basis)
+        assert ok, (e, err.max())
+
+
+@pytest.mark.parametrize("T", [1, 64])
+def test_gemm_kimi_decode_full_size_sampled(cuda_lib, T):
+    """Kimi-shaped gate_up at full size (E=384, K=7168, M=4096): every output
+    of 2 sampled experts against the oracle."""
+    torch = pytest.importorskip("torch")
+    m = cuda_lib
+    E, M, K, k = 384, 4096, 7168, 8
+    pw = pack_gpu_generated(m, 21, 0, E, M, K, chunk=4)
+    x = S.activations_bf16_np(21, T, K)
+    lg = S.uniform_logits_np(21, T, E)
+    rt = O.route(lg, k)
+    ga = np.full(E, O.act_global_scale(x), np.float32)
+    rb = m.RoutingBuffers(T, E, k)
+    m.moesq_route_permute(to_dev(lg), rb)
+    codes, scales = m.act_buffers(rb.rows_cap, K)
+    m.moesq_quantize_act(to_dev(x), T, K, rb, to_dev(ga), rb.rows_cap, codes, scales)
+    y = torch.full((rb.rows_cap, M), float("nan"), dtype=torch.bfloat16, device="cuda")
+    m.moesq_grouped_sparse_gemm(pw, codes, scales, rb.rows_cap, rb.counts, rb.row_offsets, to_dev(ga), y)
+    assert m.moesq_get_device_error()[0] == 0
+    yg_all = to_np(y)
+    ro = L.aligned_rows(rt.counts)
+    used = np.nonzero(rt.counts)[0]
+    for e in (used[0], used[-1]):
+        n = int(rt.counts[e])
+        pk = O.pack_weights(S.expert_weights_bf16_np(21, 0, int(e), M, K)[None])
+        assert (to_np(pw.values[e]) == pk.values[0]).all()
+        s0 = rt.offsets[e]
+        toks = rt.sorted_to_slot[s0:s0 + n] // k
+        c, s = O.quantize_rows_bf16(x[toks], ga[e])
+        y_ref, basis = O.grouped_gemm(pk, c, s, np.array([0, n], np.int32), ga[e:e + 1])
+        ok, err, bound, bad = gemm_tolerance_ok(yg_all[ro[e]:ro[e] + n], y_ref, basis)
+        assert ok, (e, err.max())
+
+
+def test_gemm_rejects_inconsistent_counts(cuda_lib):
+    """Counts that do not fit the aligned row offsets are refused on the
+    device (error word), nothing is written, and the context stays usable."""
+    torch = pytest.importorskip("torch")
+    m = cuda_lib
+    E, M, K = 2, 128, 256
+    pk = O.pack_weights(weights_np(9, 0, E, M, K))
+    pw = packed_from_oracle(m, pk)
+    codes, scales = m.act_buffers(256, K)
+    codes.zero_()
+    scales.zero_()
+    y = torch.zeros((256, M), dtype=torch.bfloat16, device="cuda")
+    bad_counts = to_dev(np.array([200, 5], np.int32))          # 200 rows need 256 aligned rows
+    m.moesq_grouped_sparse_gemm(pw, codes, scales, 256, bad_counts, to_dev(np.array([0, 128, 256], np.int32)),
+                                to_dev(np.ones(E, np.float32)), y)
+    st, word = m.moesq_get_device_error()
+    assert st == 5 and (word & 0xFF) == 5
+    assert float(y.float().abs().max()) == 0.0
+    ok, info = _run_isolated(m, pk, np.array([3, 4]), K, 10, 0)
+    assert ok
