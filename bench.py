@@ -1,0 +1,436 @@
+"""Benchmark of the paired-4:8 NVFP4 MoE hot path on B200.
+
+A step is one pass of the whole hot path over one batch: route + permute,
+dispatch-quantise, gate_up grouped sparse GEMM, SwiGLU + requantise, down
+grouped sparse GEMM, router-weighted combine (weight packing is offline and
+not timed).  The default workload is the 30B-class MoE layer (128 experts,
+top-8, hidden 2048, intermediate 768 -> gate_up N = 1536, T = 256 tokens,
+uniform router logits), synthetic data of the pages' distributions.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl reference]
+
+Prints one JSON line (rank 0).  `value` is the effective TFLOP/s of the
+step's two grouped GEMMs (2 * M * K per routed row, the pages' App. D.2
+definition) over all ranks; `weight_gbs` the packed expert weights the step
+reads.  Device time: CUDA events around each step on the launching stream,
+L2 flushed (256 MiB write) before every step outside the events; max over
+ranks.  `e2e`: the same metric through moesq_moe_layer_host with the step's
+inputs and output in pinned host memory (copies inside the timed region).
+`--impl reference` times the CPU oracle on a bounded token sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synthetic as S  # noqa: E402
+from grouped_gemm_moesq_b200.metrics import packed_weight_bytes  # noqa: E402
+
+METRIC = "paired-4:8 NVFP4 grouped GEMM TFLOP/s + weight GB/s vs roofline, per token count"
+
+# name -> (E, k, H, I, T, routing, kind); kind "layer" or "gemm" (route + quantise + gate_up GEMM)
+WORKLOADS = {
+    "30b_layer_t256": (128, 8, 2048, 768, 256, "uniform", "layer"),
+    "tiny_layer_t64": (8, 2, 512, 256, 64, "uniform", "layer"),
+    "kimi_layer_t1": (384, 8, 7168, 2048, 1, "uniform", "layer"),
+    "kimi_layer_t16": (384, 8, 7168, 2048, 16, "uniform", "layer"),
+    "kimi_layer_t64": (384, 8, 7168, 2048, 64, "uniform", "layer"),
+    "kimi_layer_t256": (384, 8, 7168, 2048, 256, "uniform", "layer"),
+    "kimi_layer_t4096_zipf": (384, 8, 7168, 2048, 4096, "zipf", "layer"),
+    "kimi_gateup_t1": (384, 8, 7168, 2048, 1, "uniform", "gemm"),
+    "kimi_gateup_t16": (384, 8, 7168, 2048, 16, "uniform", "gemm"),
+    "kimi_gateup_t64": (384, 8, 7168, 2048, 64, "uniform", "gemm"),
+    "kimi_gateup_t256": (384, 8, 7168, 2048, 256, "uniform", "gemm"),
+    "kimi_down_t8192_zipf": (384, 8, 2048, 7168, 8192, "zipf", "gemm_down"),
+    "30b_gateup_t256": (128, 8, 2048, 768, 256, "uniform", "gemm"),
+}
+DEFAULT_WORKLOAD = "30b_layer_t256"
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d.get("hbm_gbs", 6650.0), "measured"
+    return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        loaded = [v for v in sm if v > 0.5 * max(sm)] if sm else []
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ work accounting
+def step_work(E, k, H, I, T, counts_gu, kind):
+    """(flops, weight bytes, per-GEMM algorithmic bytes) of one step."""
+    R = T * k
+    touched = int((np.asarray(counts_gu) > 0).sum())
+    if kind == "gemm_down":
+        M, K = H, I
+        flops = 2.0 * M * K * R
+        wbytes = touched * packed_weight_bytes(M, K)
+        return flops, wbytes, {"down": wbytes + R * (K // 2 + K // 32) + R * M * 2}
+    gu_w = touched * packed_weight_bytes(2 * I, H)
+    gu_bytes = gu_w + R * (H // 2 + H // 32) + R * 2 * I * 2
+    if kind == "gemm":
+        return 2.0 * 2 * I * H * R, gu_w, {"gate_up": gu_bytes}
+    dn_w = touched * packed_weight_bytes(H, I)
+    dn_bytes = dn_w + R * (I // 2 + I // 32) + R * H * 2
+    return 2.0 * (2 * I * H + H * I) * R, gu_w + dn_w, {"gate_up": gu_bytes, "down": dn_bytes}
+
+
+def logits_for(routing, seed, T, E):
+    return S.zipf_logits_np(seed, T, E) if routing == "zipf" else S.uniform_logits_np(seed, T, E)
+
+
+# ------------------------------------------------------------------ CUDA arm
+def run_cuda(args, rank, world, local_rank):
+    import torch
+    import grouped_gemm_moesq_b200 as m
+    from grouped_gemm_moesq_b200 import build as cuda_build
+
+    if rank == 0 or not os.path.exists(cuda_build.LIB):
+        cuda_build.build()
+    m.load()
+    torch.cuda.set_device(local_rank)
+    dev = "cuda"
+    E, k, H, I, T, routing, kind = WORKLOADS[args.workload]
+    seed = 1234
+    stream = torch.cuda.current_stream()
+
+    # weights: drawn on the GPU (same bits as the host generator) and packed, 8 experts at a time
+    def make_weights(linear, M, K):
+        pw = m.PackedWeights(E, M, K)
+        for e0 in range(0, E, 8):
+            n = min(8, E - e0)
+            w = torch.stack([S.expert_weights_bf16_torch(seed, linear, e, M, K, dev) for e in range(e0, e0 + n)])
+            m.moesq_pack_weights(w, e0, n, pw)
+            del w
+        return pw
+
+    if kind == "gemm_down":
+        w_main = make_weights(1, H, I)
+        w_dn = None
+    else:
+        w_main = make_weights(0, 2 * I, H)
+        w_dn = make_weights(1, H, I) if kind == "layer" else None
+    torch.cuda.synchronize()
+
+    # per-rank batch (independent replicas: weak scaling, no data-path collective)
+    K_in = I if kind == "gemm_down" else H
+    x_np = S.activations_bf16_np(seed + 7919 * rank, T, K_in)
+    lg_np = logits_for(routing, seed + 7919 * rank, T, E)
+    x = torch.from_numpy(x_np.view(np.int16).copy()).to(dev).view(torch.bfloat16)
+    lg = torch.from_numpy(lg_np).to(dev)
+
+    rb = m.RoutingBuffers(T, E, k)
+    ga = torch.empty(E, dtype=torch.float32, device=dev)
+    gh = torch.empty(E, dtype=torch.float32, device=dev)
+    if kind == "layer":
+        ws = torch.empty(m.moesq_layer_workspace_bytes(T, k, E, H, I), dtype=torch.uint8, device=dev)
+        m.moesq_calibrate_layer(x, lg, T, k, w_main, w_dn, ga, gh, ws)
+    else:
+        m.moesq_act_global_scale(x, ga[:1])
+        ga.fill_(float(ga[:1].item()))
+    a_codes, a_scales = m.act_buffers(rb.rows_cap, K_in)
+    M_main = w_main.M
+    y_main = torch.empty(rb.rows_cap, M_main, dtype=torch.bfloat16, device=dev)
+    if kind == "layer":
+        h_codes, h_scales = m.act_buffers(rb.rows_cap, I)
+        y_dn = torch.empty(rb.rows_cap, H, dtype=torch.bfloat16, device=dev)
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+
+    def step(ev):
+        """The hot path as its ABI calls; ev: list of events recorded between them."""
+        ev[0].record(stream)
+        m.moesq_route_permute(lg, rb)
+        m.moesq_quantize_act(x, T, K_in, rb, ga, rb.rows_cap, a_codes, a_scales)
+        ev[1].record(stream)
+        m.moesq_grouped_sparse_gemm(w_main, a_codes, a_scales, rb.rows_cap, rb.counts, rb.row_offsets, ga, y_main)
+        ev[2].record(stream)
+        if kind == "layer":
+            m.moesq_swiglu_quant(y_main, I, rb, gh, h_codes, h_scales)
+            ev[3].record(stream)
+            m.moesq_grouped_sparse_gemm(w_dn, h_codes, h_scales, rb.rows_cap, rb.counts, rb.row_offsets, gh, y_dn)
+            ev[4].record(stream)
+            m.moesq_combine(y_dn, H, rb, out)
+        ev[5].record(stream)
+
+    launches_per_step = 8 if kind == "layer" else 5
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    wev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(wev)
+    torch.cuda.synchronize()
+    st, word = m.moesq_get_device_error()
+    if st != 0:
+        raise RuntimeError("device error word %#x during warm-up" % word)
+    counts = rb.counts.cpu().numpy()
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
+    t_wall0 = time.perf_counter()
+    for i in range(args.steps):
+        flush.zero_()
+        step(evs[i])
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter() - t_wall0
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    st, word = m.moesq_get_device_error()
+    if st != 0:
+        raise RuntimeError("device error word %#x in the timed region" % word)
+
+    step_ms = [e[0].elapsed_time(e[5]) for e in evs]
+    gemm1_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    parts = {"route_quant": statistics.mean(e[0].elapsed_time(e[1]) for e in evs),
+             "gemm_main": statistics.mean(gemm1_ms)}
+    if kind == "layer":
+        parts["swiglu_quant"] = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+        parts["gemm_down"] = statistics.mean(e[3].elapsed_time(e[4]) for e in evs)
+        parts["combine"] = statistics.mean(e[4].elapsed_time(e[5]) for e in evs)
+    ms = statistics.mean(step_ms)
+
+    # e2e through the public host-buffer entry point (layer workloads)
+    e2e = None
+    if kind == "layer":
+        wsh = torch.empty(m.moesq_layer_host_workspace_bytes(T, k, E, H, I), dtype=torch.uint8, device=dev)
+        xh = torch.from_numpy(x_np.view(np.int16).copy()).pin_memory()
+        lh = torch.from_numpy(lg_np).pin_memory()
+        oh = torch.empty(T, H, dtype=torch.int16).pin_memory()
+        for _ in range(args.warmup):
+            m.moesq_moe_layer_host(xh, lh, T, k, w_main, w_dn, ga, gh, oh, wsh)
+        e2e_ms = []
+        for _ in range(args.steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            m.moesq_moe_layer_host(xh, lh, T, k, w_main, w_dn, ga, gh, oh, wsh)
+            b.record(stream)
+            b.synchronize()
+            e2e_ms.append(a.elapsed_time(b))
+        e2e = {"ms_per_step": statistics.mean(e2e_ms),
+               "h2d_bytes_per_step": T * H * 2 + T * E * 4, "d2h_bytes_per_step": T * H * 2}
+
+    flops, wbytes, gemm_bytes = step_work(E, k, H, I, T, counts, kind)
+    t_max = ms
+    if world > 1:
+        tt = torch.tensor([ms, e2e["ms_per_step"] if e2e else 0.0], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_max = float(tt[0])
+        if e2e:
+            e2e["ms_per_step"] = float(tt[1])
+    return dict(kind=kind, E=E, k=k, H=H, I=I, T=T, routing=routing, ms=t_max, parts=parts, flops=flops,
+                wbytes=wbytes, gemm_bytes=gemm_bytes, e2e=e2e, clocks=clk, launches=launches_per_step * args.steps,
+                wall_s=t_wall, counts=counts)
+
+
+# ------------------------------------------------------------------ oracle (CPU) arm
+def run_oracle_sample(workload, n_tokens, seed=1234):
+    """Times the oracle on the first n_tokens tokens of the workload's batch.
+    Returns (seconds, flops of that sample)."""
+    import oracle as O
+    E, k, H, I, T, routing, kind = WORKLOADS[workload]
+    n = min(n_tokens, T)
+    K_in = I if kind == "gemm_down" else H
+    x = S.activations_bf16_np(seed, T, K_in)[:n]
+    lg = logits_for(routing, seed, T, E)[:n]
+    rt = O.route(lg, k)
+    used = np.nonzero(rt.counts)[0]
+
+    def packed(linear, M, K):
+        w = np.zeros((E, M, K), np.uint16)
+        for e in used:
+            w[e] = S.expert_weights_bf16_np(seed, linear, int(e), M, K)
+        pk = O.pack_weights(w[used])
+        full = O.Packed(np.zeros((E, M, K // 4), np.uint8), np.zeros((E, M, K // 16), np.uint8),
+                        np.zeros((E, M, K // 32), np.uint8), np.ones(E, np.float32))
+        full.values[used], full.mask[used], full.scales[used], full.gamma[used] = \
+            pk.values, pk.mask, pk.scales, pk.gamma
+        return full
+
+    ga = np.full(E, O.act_global_scale(x), np.float32)
+    if kind == "gemm_down":
+        pk = packed(1, H, I)
+        t0 = time.perf_counter()
+        rt = O.route(lg, k)
+        a_c, a_s = O.permute_quantize(x, rt, ga)
+        O.grouped_gemm(pk, a_c, a_s, rt.offsets, ga)
+        return time.perf_counter() - t0, 2.0 * H * I * n * k
+    pk_gu = packed(0, 2 * I, H)
+    if kind == "gemm":
+        t0 = time.perf_counter()
+        rt = O.route(lg, k)
+        a_c, a_s = O.permute_quantize(x, rt, ga)
+        O.grouped_gemm(pk_gu, a_c, a_s, rt.offsets, ga)
+        return time.perf_counter() - t0, 2.0 * 2 * I * H * n * k
+    pk_dn = packed(1, H, I)
+    gh = np.full(E, 64.0, np.float32)
+    t0 = time.perf_counter()
+    O.moe_layer(x, lg, k, pk_gu, pk_dn, ga, gh)
+    return time.perf_counter() - t0, 2.0 * 3 * I * H * n * k
+
+
+def oracle_sample_tokens(workload):
+    """Token sample sized for roughly 10-30 s of single-threaded oracle time."""
+    E, k, H, I, T, routing, kind = WORKLOADS[workload]
+    per_token_macs = k * (3 * I * H if kind == "layer" else 2 * I * H if kind == "gemm" else H * I)
+    return max(1, min(T, int(2.5e9 // per_token_macs)))
+
+
+# ------------------------------------------------------------------ main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    E, k, H, I, T, routing, kind = WORKLOADS[args.workload]
+    config = {"workload": args.workload, "experts": E, "top_k": k, "hidden": H, "intermediate": I,
+              "tokens_per_gpu": T, "routing": routing, "step": kind,
+              "l2": "flushed (256 MiB write) before every step, outside the timed events"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        n = oracle_sample_tokens(args.workload)
+        for _ in range(args.warmup):
+            run_oracle_sample(args.workload, max(1, n // 8))
+        secs, fl = [], 0.0
+        for _ in range(args.steps):
+            s, fl = run_oracle_sample(args.workload, n)
+            secs.append(s)
+        v = fl / statistics.mean(secs) / 1e12
+        cores = 1
+        line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(secs),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": config,
+                "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                                 "sample": "first %d of %d tokens of the workload per step" % (n, T)},
+                "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+
+    r = run_cuda(args, rank, world, local_rank)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
+    hbm_peak, peak_kind = load_peaks()
+    ms = r["ms"]
+    value = world * r["flops"] / (ms * 1e-3) / 1e12
+    weight_gbs = world * r["wbytes"] / (ms * 1e-3) / 1e9
+    gemm_key = "gemm_main"
+    gemm_ms = r["parts"][gemm_key]
+    gbytes = r["gemm_bytes"]["down" if r["kind"] == "gemm_down" else "gate_up"]
+    achieved = gbytes / (gemm_ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak, "traffic": None,
+                "kernel": "grouped_sparse_gemm (%s)" % ("down" if r["kind"] == "gemm_down" else "gate_up"),
+                "kernel_ms": gemm_ms, "peak_source": peak_kind}
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "nvfp4 (e2m1 x ue4m3 products, f32 accumulate, bf16 out)",
+            "data": "synthetic (seeded; pages' shapes and distributions)", "config": config,
+            "weight_gbs": weight_gbs, "breakdown_ms": r["parts"], "roofline": roofline,
+            "clocks": r["clocks"], "gpu_launches": r["launches"],
+            "expert_rows": {"min": int(r["counts"].min()), "max": int(r["counts"].max()),
+                            "touched": int((r["counts"] > 0).sum())}}
+    if r["e2e"]:
+        e = r["e2e"]
+        line["e2e"] = {"value": world * r["flops"] / (e["ms_per_step"] * 1e-3) / 1e12, "unit": "TFLOP/s",
+                       "h2d_bytes_per_step": e["h2d_bytes_per_step"], "d2h_bytes_per_step": e["d2h_bytes_per_step"],
+                       "ms_per_step": e["ms_per_step"]}
+    if world == 1 and not args.no_cpu_baseline:
+        n = oracle_sample_tokens(args.workload)
+        secs, fl = run_oracle_sample(args.workload, n)
+        line["cpu_baseline"] = {"value": fl / secs / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+                                "sample": "first %d of %d tokens of the workload (%.1f s)" % (n, T, secs)}
+    print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

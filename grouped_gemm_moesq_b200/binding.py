@@ -62,6 +62,7 @@ def load():
     sig = {
         "moesq_status_str": (_c.c_char_p, [_c.c_int]),
         "moesq_version": (_c.c_char_p, []),
+        "moesq_last_cuda_error": (_c.c_char_p, []),
         "moesq_get_device_error": (_c.c_int, [_vp, _P(_i32)]),
         "moesq_set_wait_timeout_ns": (None, [_c.c_uint64]),
         "moesq_weights_bytes": (_sz, [_c.c_int, _c.c_int, _c.c_int, _P(_sz)]),
@@ -96,6 +97,8 @@ def load():
 
 def _check(status: int, where: str):
     if status != 0:
+        if status == 3:
+            where = "%s [%s]" % (where, load().moesq_last_cuda_error().decode())
         raise MoesqError(status, where)
 
 
@@ -167,9 +170,12 @@ def moesq_version() -> str:
 
 
 def moesq_get_device_error(stream=None):
-    """(status, raw device word); synchronises the stream."""
+    """(status, raw device word); synchronises the stream.  A CUDA failure
+    (status 3) raises with the CUDA error text."""
     code = _i32(0)
     st = load().moesq_get_device_error(_stream(stream), ctypes.byref(code))
+    if st == 3:
+        _check(st, "moesq_get_device_error")
     return st, code.value
 
 

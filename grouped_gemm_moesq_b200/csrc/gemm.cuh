@@ -38,7 +38,7 @@ constexpr int kGemmThreads = 192;
 
 template <int TN>
 struct GemmCfg {
-  static constexpr int kStages = (TN == 128) ? 6 : 12;
+  static constexpr int kStages = (TN == 128) ? 6 : 9;
   static constexpr int kABytes = 128 * 64;       // compressed weight tile, 256 dense K
   static constexpr int kBBytes = TN * 128;       // token codes, 256 K
   static constexpr int kEBytes = 128 * 16;       // metadata
@@ -53,10 +53,11 @@ struct GemmCfg {
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kOffTab = kOffMisc + 16;
   static constexpr int kSmemBytes = kOffTab + (3 * kGemmMaxE + 1) * 4 + 1024;
-  static constexpr uint32_t kTmemCols = (TN == 128) ? 512 : 128;
+  static constexpr uint32_t kTmemCols = (TN == 128) ? 512 : 256;
   static constexpr uint32_t kColE = 2 * TN;
   static constexpr uint32_t kColSfa = 2 * TN + 4;
   static constexpr uint32_t kColSfb = 2 * TN + 12;
+  static_assert(TN == 64 || TN == 128, "token tile");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
   static_assert(kColSfb + 8 <= kTmemCols, "tensor memory");
 };
@@ -95,6 +96,9 @@ __device__ __forceinline__ Tile decode_tile(int t, int MB, int E, const int* ntp
   tl.row0 = rstart[lo] + nb * TN;
   tl.nvalid = min(TN, cnt[lo] - nb * TN);
   tl.nmma = (tl.nvalid + 15) & ~15;
+  // 32-row group of the tile inside its 128-row scale block: 0 or 2 (TN is 64
+  // or 128 and expert rows start 128-aligned), so the B-scale TMEM address
+  // moves by an even number of columns only
   tl.q = (tl.row0 & 127) >> 5;
   return tl;
 }

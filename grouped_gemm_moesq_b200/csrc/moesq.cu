@@ -29,10 +29,15 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+
 #define MOESQ_CUDA(call)                                   \
   do {                                                     \
     cudaError_t err_ = (call);                             \
-    if (err_ != cudaSuccess) return MOESQ_ERR_CUDA;        \
+    if (err_ != cudaSuccess) {                             \
+      t_last_cuda_error = err_;                            \
+      return MOESQ_ERR_CUDA;                               \
+    }                                                      \
   } while (0)
 
 #define MOESQ_TRY(call)                                    \
@@ -42,12 +47,15 @@ inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_
   } while (0)
 
 inline moesq_status last_launch() {
-  return cudaGetLastError() == cudaSuccess ? MOESQ_OK : MOESQ_ERR_CUDA;
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) return MOESQ_OK;
+  t_last_cuda_error = e;
+  return MOESQ_ERR_CUDA;
 }
 
 struct DeviceInfo {
   int sms = 0;
-  bool gemm_attr32 = false, gemm_attr128 = false;
+  bool gemm_attr64 = false, gemm_attr128 = false;
 };
 
 DeviceInfo& device_info() {
@@ -124,7 +132,7 @@ moesq_status launch_gemm(const moesq_weights* w, const uint8_t* a_codes, const u
                          int num_ctas, cudaStream_t s) {
   using C = GemmCfg<TN>;
   DeviceInfo& di = device_info();
-  bool& attr = (TN == 128) ? di.gemm_attr128 : di.gemm_attr32;
+  bool& attr = (TN == 128) ? di.gemm_attr128 : di.gemm_attr64;
   if (!attr) {
     MOESQ_CUDA(cudaFuncSetAttribute(grouped_sparse_gemm_kernel<TN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     C::kSmemBytes));
@@ -267,6 +275,10 @@ const char* moesq_status_str(moesq_status s) {
 
 const char* moesq_version(void) { return "moesq 0.1 sm_100a"; }
 
+const char* moesq_last_cuda_error(void) {
+  return t_last_cuda_error == cudaSuccess ? "no error" : cudaGetErrorString(t_last_cuda_error);
+}
+
 moesq_status moesq_get_device_error(void* stream, int32_t* device_code) {
   cudaStream_t s = as_stream(stream);
   MOESQ_CUDA(cudaStreamSynchronize(s));
@@ -391,17 +403,17 @@ moesq_status moesq_grouped_sparse_gemm(const moesq_weights* w, const uint8_t* a_
   if (!aligned(a_codes, 16) || !aligned(a_scales, 16) || !aligned(y_bf16, 2)) return MOESQ_ERR_INVALID_ARG;
   int tile_n = cfg ? cfg->tile_n : 0;
   const int num_ctas = cfg ? cfg->num_ctas : 0;
-  if (tile_n != 0 && tile_n != 32 && tile_n != 128) return MOESQ_ERR_INVALID_ARG;
+  if (tile_n != 0 && tile_n != 64 && tile_n != 128) return MOESQ_ERR_INVALID_ARG;
   if (num_ctas < 0) return MOESQ_ERR_INVALID_ARG;
   if (tile_n == 0) {
     // The counts stay on the device.  The aligned row capacity, less the
     // padding of at most 127 rows per expert, bounds the mean rows per expert.
     const int64_t rows_est = std::max<int64_t>(0, (int64_t)rows_cap - 127 * (int64_t)w->E);
-    tile_n = rows_est / w->E > 64 ? 128 : 32;
+    tile_n = rows_est / w->E > 64 ? 128 : 64;
   }
   cudaStream_t s = as_stream(stream);
-  if (tile_n == 32)
-    return launch_gemm<32>(w, a_codes, a_scales, rows_cap, counts, row_offsets, gamma_a, y_bf16, num_ctas, s);
+  if (tile_n == 64)
+    return launch_gemm<64>(w, a_codes, a_scales, rows_cap, counts, row_offsets, gamma_a, y_bf16, num_ctas, s);
   return launch_gemm<128>(w, a_codes, a_scales, rows_cap, counts, row_offsets, gamma_a, y_bf16, num_ctas, s);
 }
 

@@ -57,6 +57,10 @@ const char* moesq_status_str(moesq_status s);
 /* Library version string, e.g. "moesq 0.1 sm_100a" (static string). */
 const char* moesq_version(void);
 
+/* Text of the CUDA error behind the calling thread's most recent
+ * MOESQ_ERR_CUDA ("no error" if none); static string. */
+const char* moesq_last_cuda_error(void);
+
 /* Synchronises `stream`, then reads and clears the device error word.
  * *device_code (host) receives the raw word: 0 = none; otherwise
  * (where << 8) | kind, kind 4 = wait timeout, 5 = validation fault.
@@ -201,7 +205,7 @@ moesq_status moesq_act_global_scale(const uint16_t* x_bf16, int64_t n, float* ga
  * moesq_routing (device); they are validated on the device.
  * cfg may be NULL (defaults).                                            */
 typedef struct {
-  int32_t tile_n;      /* token rows per tile: 0 = auto, 32 or 128 */
+  int32_t tile_n;      /* token rows per tile: 0 = auto, 64 or 128 */
   int32_t num_ctas;    /* persistent CTAs: 0 = one per SM */
 } moesq_gemm_config;
 

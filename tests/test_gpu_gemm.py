@@ -44,7 +44,7 @@ def _run_isolated(m, pk, counts, K, seed, tile_n, ga_scale=1.0):
     return ok, (err.max(), np.argwhere(bad)[:5], ex)
 
 
-@pytest.mark.parametrize("tile_n", [32, 128])
+@pytest.mark.parametrize("tile_n", [64, 128])
 def test_gemm_tiny_config(cuda_lib, tile_n):
     """E=8, K=512, M=256 with the token counts of 64 tokens routed top-2."""
     E, M, K, T, k = 8, 256, 512, 64, 2
@@ -54,7 +54,7 @@ def test_gemm_tiny_config(cuda_lib, tile_n):
     assert ok, info[:2]
 
 
-@pytest.mark.parametrize("tile_n", [32, 128])
+@pytest.mark.parametrize("tile_n", [64, 128])
 @pytest.mark.parametrize("counts", [
     [0, 1, 0, 5, 0, 0, 0, 2],              # empty experts, single rows
     [129, 0, 31, 33, 1, 16, 17, 300],      # ragged: several token blocks, partial last blocks
@@ -80,7 +80,7 @@ def test_gemm_saturating_activation_scale(cuda_lib):
     """gamma_a too large: scales clip at 448 and codes at 6; still exact math."""
     E, M, K = 2, 128, 256
     pk = O.pack_weights(weights_np(7, 0, E, M, K))
-    ok, info = _run_isolated(cuda_lib, pk, np.array([20, 3]), K, 8, 32, ga_scale=64.0)
+    ok, info = _run_isolated(cuda_lib, pk, np.array([20, 3]), K, 8, 64, ga_scale=64.0)
     assert ok, info[:2]
 
 
