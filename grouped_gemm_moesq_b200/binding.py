@@ -70,6 +70,7 @@ def load():
         "moesq_rows_capacity": (_i64, [_c.c_int, _c.c_int, _c.c_int]),
         "moesq_route_workspace_bytes": (_sz, [_c.c_int, _c.c_int]),
         "moesq_route_permute": (_c.c_int, [_vp, _P(moesq_routing), _vp, _sz, _vp]),
+        "moesq_route_permute_noalloc": (_c.c_int, [_vp, _P(moesq_routing), _vp]),
         "moesq_quantize_act": (_c.c_int, [_vp, _c.c_int, _c.c_int, _P(moesq_routing), _vp, _c.c_int, _vp, _vp,
                                           _vp]),
         "moesq_act_global_scale": (_c.c_int, [_vp, _i64, _vp, _vp]),
@@ -211,6 +212,13 @@ def moesq_pack_weights(w_bf16, e_begin: int, e_count: int, out: PackedWeights, s
 def moesq_route_permute(logits, rt: RoutingBuffers, stream=None):
     _check(load().moesq_route_permute(_ptr(logits), ctypes.byref(rt.struct), _ptr(rt.workspace),
                                       rt.workspace.numel(), _stream(stream)), "moesq_route_permute")
+
+
+def moesq_route_permute_noalloc(logits, rt: RoutingBuffers, stream=None):
+    """Routing without a caller-provided workspace (static scratch inside the
+    library; T <= 16384)."""
+    _check(load().moesq_route_permute_noalloc(_ptr(logits), ctypes.byref(rt.struct), _stream(stream)),
+           "moesq_route_permute_noalloc")
 
 
 def moesq_quantize_act(x_bf16, T: int, K: int, rt, gamma, rows_cap: int, codes, scales, stream=None):

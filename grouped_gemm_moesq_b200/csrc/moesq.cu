@@ -258,6 +258,41 @@ moesq_status layer_body(const uint16_t* x, const float* logits, int T, int k, co
 
 }  // namespace
 
+// ----------------------------------------------------------------------------
+// Scratch of moesq_route_permute_noalloc: the per-block expert counts of the
+// routing kernels, for up to kNoAllocMaxT tokens and kRouteMaxE experts
+// (128 blocks x 512 experts x 4 bytes = 256 KiB).  It lives in the module's
+// global memory, so every GPU that loads the library holds it until the
+// process exits.  The name below is only a host-side handle; kernels get the
+// device address that cudaGetSymbolAddress returns for the current device.
+constexpr int kNoAllocMaxT = 16384;
+constexpr size_t kNoAllocScratchInts = (size_t)(kNoAllocMaxT / kRouteTPB) * kRouteMaxE;
+static __device__ __align__(256) int32_t g_route_scratch[kNoAllocScratchInts];
+
+namespace {
+
+// Device address of g_route_scratch on the current device, looked up once per
+// device (nullptr if the lookup fails).
+int32_t* route_scratch_device_ptr() {
+  static int32_t* ptrs[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
+    if (e != cudaSuccess) {
+      t_last_cuda_error = e;
+      return nullptr;
+    }
+    ptrs[dev] = static_cast<int32_t*>(p);
+  }
+  return ptrs[dev];
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* moesq_status_str(moesq_status s) {
@@ -512,6 +547,27 @@ moesq_status moesq_calibrate_layer(const uint16_t* x_bf16, const float* logits, 
 
 moesq_status moesq_debug_bounded_wait(uint64_t timeout_ns, void* stream) {
   debug_wait_kernel<<<1, 32, 0, as_stream(stream)>>>(timeout_ns ? timeout_ns : 1);
+  return last_launch();
+}
+
+moesq_status moesq_route_permute_noalloc(const float* logits, const moesq_routing* rt, void* stream) {
+  MOESQ_TRY(check_routing(rt));
+  if (!logits) return MOESQ_ERR_INVALID_ARG;
+  if (rt->T > kNoAllocMaxT) return MOESQ_ERR_UNSUPPORTED_SHAPE;   // beyond the static scratch
+  const int nblk = (rt->T + kRouteTPB - 1) / kRouteTPB;
+  if ((size_t)nblk * (size_t)rt->E > kNoAllocScratchInts) return MOESQ_ERR_UNSUPPORTED_SHAPE;
+  int32_t* bc = route_scratch_device_ptr();
+  if (!bc) return MOESQ_ERR_CUDA;
+  // route_topk_kernel writes every [block][expert] count the later kernels
+  // read, so the scratch needs no clearing between calls.
+  cudaStream_t s = as_stream(stream);
+  const size_t smem = (size_t)rt->E * kRouteWords * 4;
+  route_topk_kernel<<<nblk, 256, smem, s>>>(logits, rt->T, rt->E, rt->k, rt->topk_ids, rt->topk_w, bc);
+  MOESQ_TRY(last_launch());
+  route_scan_kernel<<<1, 1024, 0, s>>>(bc, nblk, rt->E, rt->counts, rt->offsets, rt->row_offsets);
+  MOESQ_TRY(last_launch());
+  route_scatter_kernel<<<nblk, 256, smem, s>>>(rt->T, rt->E, rt->k, rt->topk_ids, bc, rt->offsets, rt->row_offsets,
+                                               rt->sorted_to_slot, rt->slot_to_row);
   return last_launch();
 }
 

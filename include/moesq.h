@@ -164,6 +164,24 @@ size_t moesq_route_workspace_bytes(int T, int E);
 moesq_status moesq_route_permute(const float* logits, const moesq_routing* rt,
                                  void* workspace, size_t workspace_bytes, void* stream);
 
+/* moesq_route_permute_noalloc: the same routing as moesq_route_permute, for
+ * callers that cannot provide scratch memory -- e.g. an op slot of an
+ * inference runtime that hands the op only its inputs and outputs, or code
+ * running where allocating device memory is not allowed (a tight serving
+ * loop with a fixed memory budget).  The paper has no counterpart; this is a
+ * calling convention of this library.  Its scratch (the per-block expert
+ * counts) is a static device array inside the library, sized for at most
+ * T = 16384 tokens and E = 512 experts (256 KiB on every GPU that loads the
+ * library, held until the process exits); larger T returns
+ * MOESQ_ERR_UNSUPPORTED_SHAPE.  No memory is allocated.
+ * The first call on a device looks up the array's device address for that
+ * device (cudaGetSymbolAddress); make that first call before any stream
+ * capture.  All calls share the one array: calls that may overlap on the GPU
+ * (different streams, or different host threads) race and must be
+ * serialised by the caller.  Each call overwrites every scratch entry it
+ * reads, so nothing needs clearing between calls. */
+moesq_status moesq_route_permute_noalloc(const float* logits, const moesq_routing* rt, void* stream);
+
 /* --------------------------------------------------------- activation quant
  * Scales of an activation tensor with R rows (R a multiple of 128) and K
  * columns use the MMA scale layout [R/128][K/128][32][4][4]: the scale of
