@@ -13,9 +13,10 @@ uniform router logits), synthetic data of the pages' distributions.
 Prints one JSON line (rank 0).  `value` is the effective TFLOP/s of the
 step's two grouped GEMMs (2 * M * K per routed row, the pages' App. D.2
 definition) over all ranks; `weight_gbs` the packed expert weights the step
-reads.  Device time: CUDA events around each step on the launching stream,
-L2 flushed (256 MiB write) before every step outside the events; max over
-ranks.  `e2e`: the same metric through moesq_moe_layer_host with the step's
+reads.  Device time: the step is captured once as a CUDA graph and replayed;
+CUDA events around each replay on the launching stream, L2 flushed (256 MiB
+write) before every step outside the events; max over ranks.  The per-kernel
+breakdown replays one graph per component the same way.  `e2e`: the same metric through moesq_moe_layer_host with the step's
 inputs and output in pinned host memory (copies inside the timed region).
 `--impl reference` times the CPU oracle on a bounded token sample instead.
 """
@@ -194,34 +195,55 @@ def run_cuda(args, rank, world, local_rank):
         y_dn = torch.empty(rb.rows_cap, H, dtype=torch.bfloat16, device=dev)
         out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
 
-    def step(ev):
-        """The hot path as its ABI calls; ev: list of events recorded between them."""
-        ev[0].record(stream)
+    # the hot path as its ABI calls, one callable per component
+    def c_route_quant():
         m.moesq_route_permute(lg, rb)
         m.moesq_quantize_act(x, T, K_in, rb, ga, rb.rows_cap, a_codes, a_scales)
-        ev[1].record(stream)
+
+    def c_gemm_main():
         m.moesq_grouped_sparse_gemm(w_main, a_codes, a_scales, rb.rows_cap, rb.counts, rb.row_offsets, ga, y_main)
-        ev[2].record(stream)
-        if kind == "layer":
-            m.moesq_swiglu_quant(y_main, I, rb, gh, h_codes, h_scales)
-            ev[3].record(stream)
-            m.moesq_grouped_sparse_gemm(w_dn, h_codes, h_scales, rb.rows_cap, rb.counts, rb.row_offsets, gh, y_dn)
-            ev[4].record(stream)
-            m.moesq_combine(y_dn, H, rb, out)
-        ev[5].record(stream)
+
+    comps = [("route_quant", c_route_quant), ("gemm_main", c_gemm_main)]
+    if kind == "layer":
+        comps += [("swiglu_quant", lambda: m.moesq_swiglu_quant(y_main, I, rb, gh, h_codes, h_scales)),
+                  ("gemm_down", lambda: m.moesq_grouped_sparse_gemm(w_dn, h_codes, h_scales, rb.rows_cap, rb.counts,
+                                                                    rb.row_offsets, gh, y_dn)),
+                  ("combine", lambda: m.moesq_combine(y_dn, H, rb, out))]
+
+    def step_eager():
+        for _, f in comps:
+            f()
 
     launches_per_step = 8 if kind == "layer" else 5
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
-    wev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
     for _ in range(args.warmup):
         flush.zero_()
-        step(wev)
+        step_eager()
     torch.cuda.synchronize()
     st, word = m.moesq_get_device_error()
     if st != 0:
         raise RuntimeError("device error word %#x during warm-up" % word)
     counts = rb.counts.cpu().numpy()
+
+    # CUDA graphs: the whole step, and each component for the breakdown (the
+    # pages time CUDA-graph replays, App. D.2)
+    g_step = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step):
+        step_eager()
+    g_parts = []
+    for name, f in comps:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            f()
+        g_parts.append((name, g))
+    flush.zero_()
+    g_step.replay()
+    for _, g in g_parts:
+        g.replay()
+    torch.cuda.synchronize()
+
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
 
     if world > 1:
         import torch.distributed as dist
@@ -231,11 +253,23 @@ def run_cuda(args, rank, world, local_rank):
     clocks.start()
     time.sleep(0.3)
     t_wall0 = time.perf_counter()
+    evs = [(ev(), ev()) for _ in range(args.steps)]
     for i in range(args.steps):
         flush.zero_()
-        step(evs[i])
+        evs[i][0].record(stream)
+        g_step.replay()
+        evs[i][1].record(stream)
     torch.cuda.synchronize()
     t_wall = time.perf_counter() - t_wall0
+    # per-component breakdown, same flush discipline
+    pev = [[ev() for _ in range(len(g_parts) + 1)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        for j, (_, g) in enumerate(g_parts):
+            pev[i][j].record(stream)
+            g.replay()
+        pev[i][-1].record(stream)
+    torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
@@ -243,15 +277,9 @@ def run_cuda(args, rank, world, local_rank):
     if st != 0:
         raise RuntimeError("device error word %#x in the timed region" % word)
 
-    step_ms = [e[0].elapsed_time(e[5]) for e in evs]
-    gemm1_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    parts = {"route_quant": statistics.mean(e[0].elapsed_time(e[1]) for e in evs),
-             "gemm_main": statistics.mean(gemm1_ms)}
-    if kind == "layer":
-        parts["swiglu_quant"] = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
-        parts["gemm_down"] = statistics.mean(e[3].elapsed_time(e[4]) for e in evs)
-        parts["combine"] = statistics.mean(e[4].elapsed_time(e[5]) for e in evs)
-    ms = statistics.mean(step_ms)
+    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    parts = {name: statistics.mean(p[j].elapsed_time(p[j + 1]) for p in pev) for j, (name, _) in enumerate(g_parts)}
+    del g_step, g_parts
 
     # e2e through the public host-buffer entry point (layer workloads)
     e2e = None
@@ -357,7 +385,8 @@ def main():
     E, k, H, I, T, routing, kind = WORKLOADS[args.workload]
     config = {"workload": args.workload, "experts": E, "top_k": k, "hidden": H, "intermediate": I,
               "tokens_per_gpu": T, "routing": routing, "step": kind,
-              "l2": "flushed (256 MiB write) before every step, outside the timed events"}
+              "l2": "flushed (256 MiB write) before every step, outside the timed events",
+              "timing": "CUDA-graph replay of the step, CUDA events on the launching stream"}
 
     if args.impl == "reference":
         if rank != 0:

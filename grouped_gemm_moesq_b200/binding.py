@@ -33,7 +33,7 @@ class MoesqError(RuntimeError):
 
 class moesq_weights(ctypes.Structure):
     _fields_ = [("E", _i32), ("M", _i32), ("K", _i32), ("values", _vp), ("mask", _vp), ("scales", _vp),
-                ("global_scale", _vp), ("kmeta", _vp), ("kscales", _vp)]
+                ("global_scale", _vp), ("ktiles", _vp)]
 
 
 class moesq_routing(ctypes.Structure):
@@ -126,14 +126,13 @@ class PackedWeights:
         self.mask = torch.empty(E, M, K // 16, **u8)
         self.scales = torch.empty(E, M, K // 32, **u8)
         self.global_scale = torch.empty(E, dtype=torch.float32, device=device)
-        self.kmeta = torch.empty(E * M * K // 16, **u8)
-        self.kscales = torch.empty(E * M * K // 32, **u8)
+        self.ktiles = torch.empty(E * M * K // 32 * 11, **u8)
         self.struct = moesq_weights(E, M, K, self.values.data_ptr(), self.mask.data_ptr(), self.scales.data_ptr(),
-                                    self.global_scale.data_ptr(), self.kmeta.data_ptr(), self.kscales.data_ptr())
+                                    self.global_scale.data_ptr(), self.ktiles.data_ptr())
 
     def nbytes(self) -> int:
         return sum(t.numel() * t.element_size() for t in
-                   (self.values, self.mask, self.scales, self.global_scale, self.kmeta, self.kscales))
+                   (self.values, self.mask, self.scales, self.global_scale, self.ktiles))
 
 
 class RoutingBuffers:

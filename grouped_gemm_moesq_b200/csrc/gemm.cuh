@@ -9,11 +9,11 @@
 // inside the MMA and alpha_e in the epilogue (App. D.1).
 //
 // Design (one CTA per SM, persistent, warp-specialised):
-//   warp 0  TMA producer: per 256-wide K step it loads the compressed weight
-//           tile (128 x 64 B, 64-byte swizzle), the 128-row metadata block
-//           (2 KB) and the weight scales (1 KB) of the kernel form, the token
-//           codes (TN x 128 B, 128-byte swizzle) and their scales (1 KB) into
-//           an S-stage shared-memory ring.
+//   warp 0  producer: per 256-wide K step one bulk copy brings the weight
+//           tile of the kernel form (11 KB, contiguous: 128 x 64 B of
+//           pre-swizzled compressed values, 2 KB of metadata, 1 KB of scales);
+//           TMA brings the token codes (TN x 128 B, 128-byte swizzle) and a bulk
+//           copy their scales (1 KB) into an S-stage shared-memory ring.
 //   warp 1  MMA issuer (one thread): tcgen05.cp moves metadata and both scale
 //           blocks from shared memory into tensor memory, then two
 //           tcgen05.mma.sp.kind::mxf4nvf4.block_scale (K = 128 dense each)
@@ -30,6 +30,7 @@
 #pragma once
 #include <cuda.h>
 #include "common.cuh"
+#include "pack.cuh"
 
 namespace moesq {
 
@@ -38,16 +39,13 @@ constexpr int kGemmThreads = 192;
 
 template <int TN>
 struct GemmCfg {
-  static constexpr int kStages = (TN == 128) ? 6 : 9;
-  static constexpr int kABytes = 128 * 64;       // compressed weight tile, 256 dense K
+  static constexpr int kStages = (TN == 128) ? 7 : 10;
+  static constexpr int kWBytes = kKTileBytes;    // weight tile: A image, metadata, scales
   static constexpr int kBBytes = TN * 128;       // token codes, 256 K
-  static constexpr int kEBytes = 128 * 16;       // metadata
-  static constexpr int kSfBytes = 1024;          // 2 x (32 x 16 B)
-  static constexpr int kOffA = 0;
-  static constexpr int kOffB = kOffA + kStages * kABytes;
-  static constexpr int kOffE = kOffB + kStages * kBBytes;
-  static constexpr int kOffSfa = kOffE + kStages * kEBytes;
-  static constexpr int kOffSfb = kOffSfa + kStages * kSfBytes;
+  static constexpr int kSfBytes = 1024;          // token scales: 2 x (32 x 16 B)
+  static constexpr int kOffW = 0;
+  static constexpr int kOffB = kOffW + kStages * kWBytes;
+  static constexpr int kOffSfb = kOffB + kStages * kBBytes;
   static constexpr int kOffBar = kOffSfb + kStages * kSfBytes;
   static constexpr int kNumBars = 2 * kStages + 5;  // full, empty, acc_full[2], acc_empty[2], drain
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
@@ -58,13 +56,13 @@ struct GemmCfg {
   static constexpr uint32_t kColSfa = 2 * TN + 4;
   static constexpr uint32_t kColSfb = 2 * TN + 12;
   static_assert(TN == 64 || TN == 128, "token tile");
+  static_assert(kWBytes % 1024 == 0 && kBBytes % 1024 == 0, "1 KB aligned stages");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
   static_assert(kColSfb + 8 <= kTmemCols, "tensor memory");
 };
 
 struct GemmParams {
-  const uint8_t* kmeta;
-  const uint8_t* kscales;
+  const uint8_t* ktiles;
   const uint8_t* a_scales;
   const float* gamma_w;
   const float* gamma_a;
@@ -105,8 +103,7 @@ __device__ __forceinline__ Tile decode_tile(int t, int MB, int E, const int* ntp
 
 template <int TN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                           const GemmParams p) {
+grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const GemmParams p) {
   using C = GemmCfg<TN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -133,7 +130,6 @@ grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __gri
     mbar_init(drain_bar, 1);
     fence_barrier_init();
     misc[1] = 0;
-    prefetch_tmap(&tm_a);
     prefetch_tmap(&tm_b);
   }
   if (warp == 1) {
@@ -193,12 +189,9 @@ grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __gri
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         const Tile tl = decode_tile<TN>(t, MB, E, ntp, rstart, cnt);
         const int nbox = (tl.nmma + 31) >> 5;
-        const uint32_t bytes = C::kABytes + C::kEBytes + 2 * C::kSfBytes + nbox * 4096;
-        const int64_t wblk = (int64_t)tl.e * MB + tl.mb;
-        const uint8_t* meta = p.kmeta + wblk * KT * 2048;
-        const uint8_t* wsc = p.kscales + wblk * KB * 512;
+        const uint32_t bytes = C::kWBytes + C::kSfBytes + nbox * 4096;
+        const uint8_t* wt = p.ktiles + ((int64_t)tl.e * MB + tl.mb) * KT * C::kWBytes;
         const uint8_t* xsc = p.a_scales + (int64_t)(tl.row0 >> 7) * KB * 512;
-        const int wrow = tl.e * p.M + tl.mb * 128;
         for (int kt = 0; kt < KT; ++kt) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, p.timeout_ns, abort_flag)) {
             record_error(kWhereGemmProducer, kErrTimeout);
@@ -208,9 +201,7 @@ grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __gri
           }
           const uint32_t fb = full_bar(stage);
           mbar_arrive_expect_tx(fb, bytes);
-          tma_load_2d(sbase + C::kOffA + stage * C::kABytes, &tm_a, fb, kt * 64, wrow, pol_w);
-          bulk_load(sbase + C::kOffE + stage * C::kEBytes, meta + kt * 2048, 2048, fb, pol_w);
-          bulk_load(sbase + C::kOffSfa + stage * C::kSfBytes, wsc + kt * 1024, 1024, fb, pol_w);
+          bulk_load(sbase + C::kOffW + stage * C::kWBytes, wt + (int64_t)kt * C::kWBytes, C::kWBytes, fb, pol_w);
           bulk_load(sbase + C::kOffSfb + stage * C::kSfBytes, xsc + kt * 1024, 1024, fb, pol_x);
           for (int i = 0; i < nbox; ++i)
             tma_load_2d(sbase + C::kOffB + stage * C::kBBytes + i * 4096, &tm_b, fb, kt * 128, tl.row0 + 32 * i,
@@ -253,10 +244,10 @@ grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __gri
             break;
           }
           tc_fence_after();
-          const uint32_t sa = sbase + C::kOffA + stage * C::kABytes;
+          const uint32_t sa = sbase + C::kOffW + stage * C::kWBytes;
           const uint32_t sb = sbase + C::kOffB + stage * C::kBBytes;
-          const uint32_t se = sbase + C::kOffE + stage * C::kEBytes;
-          const uint32_t ssa = sbase + C::kOffSfa + stage * C::kSfBytes;
+          const uint32_t se = sa + kKTileMeta;
+          const uint32_t ssa = sa + kKTileScales;
           const uint32_t ssb = sbase + C::kOffSfb + stage * C::kSfBytes;
           tc_cp_128x128b(tmem + C::kColE, smem_desc(se, 16, 128, 0));
           tc_cp_32x128b_x4(tmem + C::kColSfa, smem_desc(ssa, 16, 128, 0));

@@ -106,10 +106,8 @@ moesq_status check_weights(const moesq_weights* w) {
   if (!w) return MOESQ_ERR_INVALID_ARG;
   if (w->E < 1 || w->E > kGemmMaxE || w->M < 128 || w->K < 256) return MOESQ_ERR_UNSUPPORTED_SHAPE;
   if (w->M % 128 || w->K % 256) return MOESQ_ERR_UNSUPPORTED_SHAPE;
-  if (!w->values || !w->mask || !w->scales || !w->global_scale || !w->kmeta || !w->kscales)
-    return MOESQ_ERR_INVALID_ARG;
-  if (!aligned(w->values, 16) || !aligned(w->kmeta, 16) || !aligned(w->kscales, 16) || !aligned(w->mask, 2) ||
-      !aligned(w->global_scale, 4))
+  if (!w->values || !w->mask || !w->scales || !w->global_scale || !w->ktiles) return MOESQ_ERR_INVALID_ARG;
+  if (!aligned(w->values, 16) || !aligned(w->ktiles, 16) || !aligned(w->mask, 2) || !aligned(w->global_scale, 4))
     return MOESQ_ERR_INVALID_ARG;
   if ((int64_t)w->E * w->M >= (int64_t)1 << 31) return MOESQ_ERR_UNSUPPORTED_SHAPE;
   return MOESQ_OK;
@@ -138,15 +136,11 @@ moesq_status launch_gemm(const moesq_weights* w, const uint8_t* a_codes, const u
                                     C::kSmemBytes));
     attr = true;
   }
-  CUtensorMap tma, tmb;
-  if (!make_tmap(&tma, w->values, (uint64_t)w->K / 4, (uint64_t)w->E * w->M, 64, 128,
-                 CU_TENSOR_MAP_SWIZZLE_64B))
-    return MOESQ_ERR_CUDA;
+  CUtensorMap tmb;
   if (!make_tmap(&tmb, a_codes, (uint64_t)w->K / 2, (uint64_t)rows_cap, 128, 32, CU_TENSOR_MAP_SWIZZLE_128B))
     return MOESQ_ERR_CUDA;
   GemmParams p;
-  p.kmeta = w->kmeta;
-  p.kscales = w->kscales;
+  p.ktiles = w->ktiles;
   p.a_scales = a_scales;
   p.gamma_w = w->global_scale;
   p.gamma_a = gamma_a;
@@ -159,7 +153,7 @@ moesq_status launch_gemm(const moesq_weights* w, const uint8_t* a_codes, const u
   p.rows_cap = rows_cap;
   p.timeout_ns = g_timeout_ns;
   const int grid = num_ctas > 0 ? num_ctas : di.sms;
-  grouped_sparse_gemm_kernel<TN><<<grid, kGemmThreads, C::kSmemBytes, s>>>(tma, tmb, p);
+  grouped_sparse_gemm_kernel<TN><<<grid, kGemmThreads, C::kSmemBytes, s>>>(tmb, p);
   return last_launch();
 }
 
@@ -329,9 +323,9 @@ void moesq_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns = ns ? ns : 1; }
 
 size_t moesq_weights_bytes(int E, int M, int K, size_t* per_tensor) {
   const size_t emk = (size_t)E * M * K;
-  size_t t[6] = {emk / 4, emk / 16, emk / 32, (size_t)E * 4, emk / 16, emk / 32};
+  size_t t[5] = {emk / 4, emk / 16, emk / 32, (size_t)E * 4, emk / 32 * 11};
   size_t sum = 0;
-  for (int i = 0; i < 6; ++i) {
+  for (int i = 0; i < 5; ++i) {
     if (per_tensor) per_tensor[i] = t[i];
     sum += align256(t[i]);
   }
@@ -355,7 +349,7 @@ moesq_status moesq_pack_weights(const uint16_t* w_bf16, int e_begin, int e_count
   MOESQ_TRY(last_launch());
   pack_gamma_kernel<<<(e_count + 255) / 256, 256, 0, s>>>(gamma, e_count);
   MOESQ_TRY(last_launch());
-  PackOut po{out->values, out->mask, out->scales, out->global_scale, out->kmeta, out->kscales};
+  PackOut po{out->values, out->mask, out->scales, out->global_scale, out->ktiles};
   const int64_t n_blocks = (int64_t)e_count * M * (K / 32);
   pack_blocks_kernel<<<grid_for(n_blocks, 256, sms), 256, 0, s>>>(w_bf16, e_begin, n_blocks, M, K, po);
   return last_launch();
@@ -382,7 +376,7 @@ moesq_status moesq_route_permute(const float* logits, const moesq_routing* rt, v
   const int nblk = (rt->T + kRouteTPB - 1) / kRouteTPB;
   int32_t* bc = static_cast<int32_t*>(workspace);
   const size_t smem = (size_t)rt->E * kRouteWords * 4;
-  route_topk_kernel<<<nblk, 256, smem, s>>>(logits, rt->T, rt->E, rt->k, rt->topk_ids, rt->topk_w, bc);
+  route_topk_kernel<<<nblk, 1024, smem, s>>>(logits, rt->T, rt->E, rt->k, rt->topk_ids, rt->topk_w, bc);
   MOESQ_TRY(last_launch());
   route_scan_kernel<<<1, 1024, 0, s>>>(bc, nblk, rt->E, rt->counts, rt->offsets, rt->row_offsets);
   MOESQ_TRY(last_launch());
@@ -562,7 +556,7 @@ moesq_status moesq_route_permute_noalloc(const float* logits, const moesq_routin
   // read, so the scratch needs no clearing between calls.
   cudaStream_t s = as_stream(stream);
   const size_t smem = (size_t)rt->E * kRouteWords * 4;
-  route_topk_kernel<<<nblk, 256, smem, s>>>(logits, rt->T, rt->E, rt->k, rt->topk_ids, rt->topk_w, bc);
+  route_topk_kernel<<<nblk, 1024, smem, s>>>(logits, rt->T, rt->E, rt->k, rt->topk_ids, rt->topk_w, bc);
   MOESQ_TRY(last_launch());
   route_scan_kernel<<<1, 1024, 0, s>>>(bc, nblk, rt->E, rt->counts, rt->offsets, rt->row_offsets);
   MOESQ_TRY(last_launch());

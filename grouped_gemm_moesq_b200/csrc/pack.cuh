@@ -5,7 +5,7 @@
 // (paper App. A Eq. 6 pattern set; model card "exactly 2 pairs are kept").
 // Scales: paper Sec. 3.4 Eq. 5 on the masked weights; values: Eq. 3.
 // Outputs the storage form of the model card (values / mask / scales /
-// gamma) and the kernel form read by the grouped GEMM (kmeta / kscales).
+// gamma) and the kernel form read by the grouped GEMM (ktiles).
 #pragma once
 #include "common.cuh"
 
@@ -65,19 +65,23 @@ __global__ void pack_gamma_kernel(float* __restrict__ gamma, int n) {
   if (i < n) gamma[i] = nvfp4_global_scale(gamma[i]);   // gamma[i] holds amax here
 }
 
+// Kernel-form tile of 128 weight rows x 256 dense K (see include/moesq.h).
+constexpr int kKTileBytes = 11264;
+constexpr int kKTileMeta = 8192;
+constexpr int kKTileScales = 10240;
+
 struct PackOut {
   uint8_t* values;    // [E][M][K/4]
   uint8_t* mask;      // [E][M][K/16]
   uint8_t* scales;    // [E][M][K/32]
   const float* gamma; // [E]
-  uint8_t* kmeta;     // [E][M/128][K/256][128][16]
-  uint8_t* kscales;   // [E][M/128][K/128][512]
+  uint8_t* ktiles;    // [E][M/128][K/256][kKTileBytes]
 };
 
 // Pass 2: one thread per 32-element block (4 groups, 16 kept values).
 __global__ void pack_blocks_kernel(const uint16_t* __restrict__ w, int e_begin, int64_t n_blocks, int M,
                                    int K, PackOut out) {
-  const int nb_row = K / 32, KT = K / 256, KB = K / 128, MB = M / 128;
+  const int nb_row = K / 32, KT = K / 256, MB = M / 128;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < n_blocks; t += stride) {
     const int b = (int)(t % nb_row);
@@ -125,7 +129,8 @@ __global__ void pack_blocks_kernel(const uint16_t* __restrict__ w, int e_begin, 
     *reinterpret_cast<uint16_t*>(out.mask + row * (K / 16) + (int64_t)b * 2) = mk;
     out.scales[row * nb_row + b] = (uint8_t)code;
 
-    // kernel form: metadata nibble = i0 | i1 << 2 of the two kept pair indices
+    // kernel form, tile (e, mb, kt): swizzled values, metadata nibbles
+    // i0 | i1 << 2 of the two kept pair indices, scales in the MMA layout
     uint32_t meta = 0;
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
@@ -134,13 +139,13 @@ __global__ void pack_blocks_kernel(const uint16_t* __restrict__ w, int e_begin, 
       const uint32_t i1 = 31 - __clz(bits);
       meta |= (i0 | (i1 << 2)) << (4 * g);
     }
-    const int mb = m >> 7, i = m & 127;
-    const int kt = b >> 3;
-    const int64_t mo = ((((int64_t)e * MB + mb) * KT + kt) * 128 + i) * 16 + (b & 7) * 2;
-    *reinterpret_cast<uint16_t*>(out.kmeta + mo) = (uint16_t)meta;
-    const int kb = b >> 2, s = b & 3;
-    const int64_t so = (((int64_t)e * MB + mb) * KB + kb) * 512 + (i & 31) * 16 + (i >> 5) * 4 + s;
-    out.kscales[so] = (uint8_t)code;
+    const int mb = m >> 7, r = m & 127;
+    const int kt = b >> 3, bt = b & 7;            // 32-block within the 256-wide K tile
+    uint8_t* tile = out.ktiles + (((int64_t)e * MB + mb) * KT + kt) * kKTileBytes;
+    const int chunk = (bt >> 1) ^ ((r >> 1) & 3);  // 16-byte chunk after the swizzle
+    *reinterpret_cast<uint2*>(tile + r * 64 + chunk * 16 + (bt & 1) * 8) = vbytes;
+    *reinterpret_cast<uint16_t*>(tile + kKTileMeta + r * 16 + bt * 2) = (uint16_t)meta;
+    tile[kKTileScales + (bt >> 2) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (bt & 3)] = (uint8_t)code;
   }
 }
 

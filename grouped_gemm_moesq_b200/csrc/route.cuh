@@ -13,12 +13,26 @@ constexpr int kRouteWords = kRouteTPB / 32;
 constexpr int kRouteMaxE = 512;
 constexpr int kRouteMaxPerLane = kRouteMaxE / 32;
 
-// K1: one warp per token: top-k (descending logit, ties to the lower id),
-// softmax gate weights over all E logits, and the block's per-expert token
-// bitmaps -> per-block counts [nblk][E].
-__global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
-                                                         int32_t* __restrict__ topk_ids, float* __restrict__ topk_w,
-                                                         int32_t* __restrict__ block_counts) {
+// Order-preserving map of a finite float to uint32 (-0 maps like +0; NaN
+// maps to 0 and is never chosen while a number is left).
+__device__ __forceinline__ uint32_t ordered_bits(float v) {
+  if (v != v) return 0u;
+  const uint32_t u = __float_as_uint(v == 0.0f ? 0.0f : v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float from_ordered_bits(uint32_t o) {
+  return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
+}
+
+// K1: one warp per token (32 warps, 4 tokens each, per 128-token block):
+// top-k by descending logit with ties to the lower id, softmax gate weights
+// over all E logits, and the block's per-expert token bitmaps -> per-block
+// counts [nblk][E].  Each pick is two warp reductions (max of the ordered
+// value, then min of the ids holding it).
+__global__ void __launch_bounds__(1024) route_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                          int32_t* __restrict__ topk_ids, float* __restrict__ topk_w,
+                                                          int32_t* __restrict__ block_counts) {
   extern __shared__ uint32_t bitmap[];                 // [E][kRouteWords]
   for (int i = threadIdx.x; i < E * kRouteWords; i += blockDim.x) bitmap[i] = 0;
   __syncthreads();
@@ -28,51 +42,48 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
     const int t = blockIdx.x * kRouteTPB + tl;
     if (t >= T) break;
     const float* lr = logits + (size_t)t * E;
-    float v[kRouteMaxPerLane];
+    uint32_t o[kRouteMaxPerLane];          // ordered bits; the logit is recovered exactly from them
     float mx = -INFINITY;
 #pragma unroll
     for (int i = 0; i < kRouteMaxPerLane; ++i) {
       const int e = lane + 32 * i;
-      v[i] = (i < per_lane && e < E) ? lr[e] : -INFINITY;
-      mx = fmaxf(mx, v[i]);
+      const float x = (i < per_lane && e < E) ? __ldg(lr + e) : -INFINITY;
+      o[i] = (i < per_lane && e < E) ? ordered_bits(x) : 0u;
+      mx = fmaxf(mx, x);
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
     float z = 0.0f;
 #pragma unroll
     for (int i = 0; i < kRouteMaxPerLane; ++i) {
       const int e = lane + 32 * i;
-      if (i < per_lane && e < E) z += expf(v[i] - mx);
+      if (i < per_lane && e < E) z += expf(from_ordered_bits(o[i]) - mx);
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
     uint32_t taken = 0;
     for (int j = 0; j < k; ++j) {
-      float bv = -INFINITY;
+      uint32_t bo = 0;
       int be = 0x7fffffff;
 #pragma unroll
       for (int i = 0; i < kRouteMaxPerLane; ++i) {
         const int e = lane + 32 * i;
-        if (i < per_lane && e < E && !(taken >> i & 1u) && (v[i] > bv || (v[i] == bv && e < be))) {
-          bv = v[i];
+        if (i < per_lane && e < E && !(taken >> i & 1u) && o[i] > bo) {   // ids ascend with i: > keeps the lowest
+          bo = o[i];
           be = e;
         }
       }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-        if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
-      }
-      if (be >= E) {                       // only NaN logits leave no candidate
+      const uint32_t best = __reduce_max_sync(0xffffffffu, bo);
+      const int win = __reduce_min_sync(0xffffffffu, (bo == best && be < E) ? be : 0x7fffffff);
+      if (win >= E) {                      // only NaN logits leave no candidate
         if (lane == 0) record_error(kWhereRoute, kErrFault);
-        be = j;
+        break;
       }
-      if ((be & 31) == lane) taken |= 1u << (be >> 5);
-      if (lane == 0) {
-        topk_ids[(size_t)t * k + j] = be;
-        topk_w[(size_t)t * k + j] = __fdiv_rn(expf(bv - mx), z);
-        atomicOr(&bitmap[be * kRouteWords + (tl >> 5)], 1u << (tl & 31));
+      if ((win & 31) == lane) {
+        taken |= 1u << (win >> 5);
+        topk_ids[(size_t)t * k + j] = win;
+        topk_w[(size_t)t * k + j] = __fdiv_rn(expf(from_ordered_bits(bo) - mx), z);
+        atomicOr(&bitmap[win * kRouteWords + (tl >> 5)], 1u << (tl & 31));
       }
     }
   }

@@ -86,26 +86,33 @@ void moesq_set_wait_timeout_ns(uint64_t ns);
  *                        Eq. 5 (dequantised weight = code * scale / gamma)
  * Kernel form (derived at pack time, the "kernel's own layout" the model
  * card's loader builds; read only by moesq_grouped_sparse_gemm):
- *   kmeta   [E][M/128][K/256][128][16]  sparse-MMA metadata: for row i of a
- *           128-row block and a 256-wide K tile, byte b holds chunks 2b (low
- *           nibble) and 2b+1; a chunk's nibble is i0 | i1 << 2, the indices
- *           i0 < i1 of its two kept pairs
- *   kscales [E][M/128][K/128][32][4][4] the UE4M3 scales of rows 32a+b and
- *           K sub-blocks s of a 128-wide K block at byte b*16 + a*4 + s
- * values is also the compressed left operand of the sparse MMA as is.    */
+ *   ktiles  [E][M/128][K/256][11264]  one contiguous tile per 128 weight rows
+ *           and 256 dense K, copied to shared memory as is:
+ *     bytes [0, 8192)      the tile's 128 rows of `values` (64 B each), row r
+ *                          at r*64 with its 16-byte chunk c stored in chunk
+ *                          position c ^ ((r >> 1) & 3) (the 64-byte swizzle the
+ *                          tensor-core descriptor reads)
+ *     bytes [8192, 10240)  sparse-MMA metadata, 16 B per row: byte b holds
+ *                          chunks 2b (low nibble) and 2b+1; a chunk's nibble
+ *                          is i0 | i1 << 2, the indices i0 < i1 of its two
+ *                          kept pairs
+ *     bytes [10240, 11264) the UE4M3 scales of the two 128-wide K halves, 512 B
+ *                          each: the scale of row 32a+b and K sub-block s at
+ *                          byte b*16 + a*4 + s
+ * The kernel form holds the same 11*M*K/32 bytes per expert as the storage
+ * form, rearranged so that one K step of the GEMM is one sequential read. */
 typedef struct {
   int32_t E, M, K;
   uint8_t* values;
   uint8_t* mask;
   uint8_t* scales;
   float* global_scale;
-  uint8_t* kmeta;
-  uint8_t* kscales;
+  uint8_t* ktiles;
 } moesq_weights;
 
-/* Bytes of each weight tensor: per_tensor[0..5] (host, may be NULL) =
- * values, mask, scales, global_scale, kmeta, kscales.  Returns the sum
- * (each tensor rounded up to 256 bytes). */
+/* Bytes of each weight tensor: per_tensor[0..4] (host, may be NULL) =
+ * values, mask, scales, global_scale, ktiles.  Returns the sum (each tensor
+ * rounded up to 256 bytes). */
 size_t moesq_weights_bytes(int E, int M, int K, size_t* per_tensor);
 
 /* moesq_pack_weights: bf16 expert weights -> paired-4:8 NVFP4, for experts

@@ -65,8 +65,7 @@ def packed_from_oracle(m, pk):
     pw.mask.copy_(torch.from_numpy(pk.mask))
     pw.scales.copy_(torch.from_numpy(pk.scales))
     pw.global_scale.copy_(torch.from_numpy(pk.gamma))
-    pw.kmeta.copy_(torch.from_numpy(L.mask_to_kmeta(pk.mask)))
-    pw.kscales.copy_(torch.from_numpy(L.weight_scales_to_kscales(pk.scales)))
+    pw.ktiles.copy_(torch.from_numpy(L.storage_to_ktiles(pk.values, pk.mask, pk.scales)))
     torch.cuda.synchronize()
     return pw
 

@@ -1,12 +1,14 @@
 """Host-side transforms between the storage form and the kernel layouts that
 include/moesq.h defines (test helpers; numpy only).
 
-* kmeta   [E][M/128][K/256][128][16]: byte b of row i holds the metadata of
-          chunks 2b (low nibble) and 2b+1; a chunk nibble is i0 | i1 << 2 of
-          its two kept pair indices.
-* kscales [E][M/128][K/128][32][4][4] and the activation scale layout
-          [R/128][K/128][32][4][4]: scale of row 32a+b (of a 128-row block),
-          sub-block s of a 128-wide K block, at byte b*16 + a*4 + s.
+* ktiles  [E][M/128][K/256][11264]: per tile the 128 rows of values (64 B
+          each, 16-byte chunk c of row r at chunk c ^ ((r >> 1) & 3)), then
+          the metadata [128][16] (byte b of row i holds chunks 2b, 2b+1; a chunk
+          nibble is i0 | i1 << 2 of its two kept pair indices), then the
+          scales of the two 128-wide K halves in the MMA scale layout.
+* MMA scale layout (weights per tile, activations [R/128][K/128][512]):
+          scale of row 32a+b (of a 128-row block), sub-block s of a 128-wide K
+          block, at byte b*16 + a*4 + s.
 * aligned row space: expert e owns rows row_offsets[e] + [0, counts[e]).
 """
 import numpy as np
@@ -46,6 +48,38 @@ def scales_to_mma(sc: np.ndarray) -> np.ndarray:
     # [R/128, 4(a), 32(b), K/128, 4(s)] -> [R/128, K/128, 32(b), 4(a), 4(s)]
     t = sc.reshape(R // 128, 4, 32, S // 4, 4).transpose(0, 3, 2, 1, 4)
     return np.ascontiguousarray(t).reshape(-1)
+
+
+def storage_to_ktiles(values: np.ndarray, mask: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """Storage form [E, M, *] -> kernel-form tiles (flat uint8)."""
+    E, M, K4 = values.shape
+    K = 4 * K4
+    MB, KT = M // 128, K // 256
+    v = values.reshape(E, MB, 128, KT, 4, 16).transpose(0, 1, 3, 2, 4, 5)   # [E,MB,KT,r,c,16]
+    r = np.arange(128)[:, None]
+    c = np.arange(4)[None, :]
+    img = np.empty_like(v)
+    img[:, :, :, r, c ^ ((r >> 1) & 3), :] = v[:, :, :, r, c, :]
+    meta = mask_to_kmeta(mask).reshape(E, MB, KT, 128 * 16)
+    sc = weight_scales_to_kscales(scales).reshape(E, MB, KT, 1024)
+    out = np.concatenate([img.reshape(E, MB, KT, 8192), meta, sc], axis=-1)
+    return np.ascontiguousarray(out).reshape(-1)
+
+
+def ktiles_to_storage(flat: np.ndarray, E: int, M: int, K: int):
+    """Kernel-form tiles -> (values, mask, scales) of the storage form."""
+    MB, KT = M // 128, K // 256
+    t = flat.reshape(E, MB, KT, 11264)
+    img = t[..., :8192].reshape(E, MB, KT, 128, 4, 16)
+    r = np.arange(128)[:, None]
+    c = np.arange(4)[None, :]
+    v = img[:, :, :, r, c ^ ((r >> 1) & 3), :]                              # [E,MB,KT,r,c,16]
+    values = v.transpose(0, 1, 3, 2, 4, 5).reshape(E, M, K // 4)
+    meta = t[..., 8192:10240].reshape(-1)
+    mask = kmeta_to_mask(np.ascontiguousarray(meta), E, M, K)
+    sc = np.ascontiguousarray(t[..., 10240:]).reshape(-1)
+    scales = kscales_to_weight_scales(sc, E, M, K)
+    return np.ascontiguousarray(values), mask, scales
 
 
 def mma_to_scales(flat: np.ndarray, R: int, K: int) -> np.ndarray:

@@ -47,10 +47,11 @@ def test_host_only_helpers(lib):
     import grouped_gemm_moesq_b200 as m
     m.load()
     # Eq. 7 storage: values K/4 + mask K/16 + scales K/32 per row, plus kernel form
-    per = (ctypes.c_size_t * 6)()
+    per = (ctypes.c_size_t * 5)()
     m.load().moesq_weights_bytes(384, 4096, 7168, per)
     assert per[0] == 384 * 4096 * 7168 // 4 and per[1] == per[0] // 4 and per[2] == per[0] // 8
     assert per[0] + per[1] + per[2] == 11 * 384 * 4096 * 7168 // 32
+    assert per[4] == per[0] + per[1] + per[2]          # kernel form: the same bytes, tiled
     assert m.moesq_rows_capacity(1, 8, 384) == 1024
     assert m.moesq_rows_capacity(8192, 8, 384) % 128 == 0
     assert m.moesq_rows_capacity(8192, 8, 384) >= 8192 * 8 + 127 * 384

@@ -17,8 +17,9 @@ def _check_pack(pw, pk, E, M, K):
     assert (to_np(pw.mask) == pk.mask).all()
     assert (to_np(pw.scales) == pk.scales).all()
     assert (to_np(pw.global_scale).view(np.uint32) == pk.gamma.view(np.uint32)).all()
-    assert (to_np(pw.kmeta) == L.mask_to_kmeta(pk.mask)).all()
-    assert (to_np(pw.kscales) == L.weight_scales_to_kscales(pk.scales)).all()
+    assert (to_np(pw.ktiles) == L.storage_to_ktiles(pk.values, pk.mask, pk.scales)).all()
+    v, mk, sc = L.ktiles_to_storage(to_np(pw.ktiles), E, M, K)
+    assert (v == pk.values).all() and (mk == pk.mask).all() and (sc == pk.scales).all()
 
 
 @pytest.mark.parametrize("E,M,K", [(8, 256, 512), (3, 128, 256)])
@@ -42,8 +43,8 @@ def test_pack_30b_class_sampled_experts(cuda_lib):
         assert (to_np(pw.mask[e]) == pk.mask[0]).all()
         assert (to_np(pw.scales[e]) == pk.scales[0]).all()
         assert to_np(pw.global_scale)[e] == pk.gamma[0]
-        per = M * K // 16
-        assert (to_np(pw.kmeta[e * per:(e + 1) * per]) == L.mask_to_kmeta(pk.mask)).all()
+        per = M * K // 32 * 11
+        assert (to_np(pw.ktiles[e * per:(e + 1) * per]) == L.storage_to_ktiles(pk.values, pk.mask, pk.scales)).all()
 
 
 # ---------------------------------------------------------------- routing
