@@ -15,8 +15,8 @@ step's two grouped GEMMs (2 * M * K per routed row, the pages' App. D.2
 definition) over all ranks; `weight_gbs` the packed expert weights the step
 reads.  Device time: the step is captured once as a CUDA graph and replayed;
 CUDA events around each replay on the launching stream, L2 flushed (256 MiB
-write) before every step outside the events; max over ranks.  The per-kernel
-breakdown replays one graph per component the same way.  `e2e`: the same metric through moesq_moe_layer_host with the step's
+write) before every step outside the events; max over ranks.  Event nodes
+inside the graph give the per-kernel breakdown of the same replays.  `e2e`: the same metric through moesq_moe_layer_host with the step's
 inputs and output in pinned host memory (copies inside the timed region).
 `--impl reference` times the CPU oracle on a bounded token sample instead.
 """
@@ -54,7 +54,7 @@ WORKLOADS = {
     "kimi_gateup_t16": (384, 8, 7168, 2048, 16, "uniform", "gemm"),
     "kimi_gateup_t64": (384, 8, 7168, 2048, 64, "uniform", "gemm"),
     "kimi_gateup_t256": (384, 8, 7168, 2048, 256, "uniform", "gemm"),
-    "kimi_down_t8192_zipf": (384, 8, 2048, 7168, 8192, "zipf", "gemm_down"),
+    "kimi_down_t8192_zipf": (384, 8, 7168, 2048, 8192, "zipf", "gemm_down"),
     "30b_gateup_t256": (128, 8, 2048, 768, 256, "uniform", "gemm"),
 }
 DEFAULT_WORKLOAD = "30b_layer_t256"
@@ -225,21 +225,30 @@ def run_cuda(args, rank, world, local_rank):
         raise RuntimeError("device error word %#x during warm-up" % word)
     counts = rb.counts.cpu().numpy()
 
-    # CUDA graphs: the whole step, and each component for the breakdown (the
-    # pages time CUDA-graph replays, App. D.2)
-    g_step = torch.cuda.CUDAGraph()
+    # One CUDA graph per step (the pages time CUDA-graph replays, App. D.2),
+    # with external event-record nodes between the components: the same
+    # replays give the per-kernel breakdown on the launching stream.
+    from cuda.bindings import runtime as cudart
+
+    def cu_event():
+        err, e = cudart.cudaEventCreate()
+        assert err == cudart.cudaError_t.cudaSuccess
+        return e
+
+    cev = [cu_event() for _ in range(len(comps) + 1)]
+    g_step = torch.cuda.CUDAGraph()          # the timed step: kernels only
     with torch.cuda.graph(g_step):
         step_eager()
-    g_parts = []
-    for name, f in comps:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
+    g_prof = torch.cuda.CUDAGraph()          # the same kernels with event nodes between them
+    with torch.cuda.graph(g_prof):
+        cs = torch.cuda.current_stream().cuda_stream
+        for j, (_, f) in enumerate(comps):
+            cudart.cudaEventRecordWithFlags(cev[j], cs, cudart.cudaEventRecordExternal)
             f()
-        g_parts.append((name, g))
+        cudart.cudaEventRecordWithFlags(cev[-1], cs, cudart.cudaEventRecordExternal)
     flush.zero_()
     g_step.replay()
-    for _, g in g_parts:
-        g.replay()
+    g_prof.replay()
     torch.cuda.synchronize()
 
     def ev():
@@ -254,6 +263,7 @@ def run_cuda(args, rank, world, local_rank):
     time.sleep(0.3)
     t_wall0 = time.perf_counter()
     evs = [(ev(), ev()) for _ in range(args.steps)]
+    part_ms = {name: [] for name, _ in comps}
     for i in range(args.steps):
         flush.zero_()
         evs[i][0].record(stream)
@@ -261,15 +271,14 @@ def run_cuda(args, rank, world, local_rank):
         evs[i][1].record(stream)
     torch.cuda.synchronize()
     t_wall = time.perf_counter() - t_wall0
-    # per-component breakdown, same flush discipline
-    pev = [[ev() for _ in range(len(g_parts) + 1)] for _ in range(args.steps)]
-    for i in range(args.steps):
+    for i in range(args.steps):                 # per-kernel breakdown, same flush discipline
         flush.zero_()
-        for j, (_, g) in enumerate(g_parts):
-            pev[i][j].record(stream)
-            g.replay()
-        pev[i][-1].record(stream)
-    torch.cuda.synchronize()
+        g_prof.replay()
+        torch.cuda.synchronize()
+        for j, (name, _) in enumerate(comps):
+            err, dt = cudart.cudaEventElapsedTime(cev[j], cev[j + 1])
+            assert err == cudart.cudaError_t.cudaSuccess, err
+            part_ms[name].append(dt)
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
@@ -278,8 +287,10 @@ def run_cuda(args, rank, world, local_rank):
         raise RuntimeError("device error word %#x in the timed region" % word)
 
     ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
-    parts = {name: statistics.mean(p[j].elapsed_time(p[j + 1]) for p in pev) for j, (name, _) in enumerate(g_parts)}
-    del g_step, g_parts
+    parts = {name: statistics.mean(v) for name, v in part_ms.items()}
+    del g_step, g_prof
+    for e in cev:
+        cudart.cudaEventDestroy(e)
 
     # e2e through the public host-buffer entry point (layer workloads)
     e2e = None

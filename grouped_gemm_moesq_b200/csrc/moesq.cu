@@ -222,6 +222,38 @@ moesq_routing routing_of(const LayerWs& w, int T, int E, int k) {
   return rt;
 }
 
+// Launches the routing kernels for logits [T][E] into rt, with the per-block
+// counts in bc (nblk x E int32).  PL = logits per lane of a token's warp.
+template <int PL>
+moesq_status route_launch_pl(const float* logits, const moesq_routing* rt, int32_t* bc, cudaStream_t s) {
+  const int nblk = (rt->T + kRouteTPB - 1) / kRouteTPB;
+  const size_t smem = (size_t)rt->E * kRouteWords * 4;
+  if (nblk == 1) {                      // one token block: fused single-CTA path
+    route_small_kernel<PL><<<1, 1024, smem, s>>>(logits, rt->T, rt->E, rt->k, rt->topk_ids, rt->topk_w, rt->counts,
+                                                 rt->offsets, rt->row_offsets, rt->sorted_to_slot, rt->slot_to_row);
+    return last_launch();
+  }
+  route_topk_kernel<PL><<<(rt->T + 7) / 8, 256, 0, s>>>(logits, rt->T, rt->E, rt->k, rt->topk_ids, rt->topk_w);
+  MOESQ_TRY(last_launch());
+  route_count_kernel<<<nblk, 256, smem, s>>>(rt->T, rt->E, rt->k, rt->topk_ids, bc);
+  MOESQ_TRY(last_launch());
+  route_scan_kernel<<<1, 1024, 0, s>>>(bc, nblk, rt->E, rt->counts, rt->offsets, rt->row_offsets);
+  MOESQ_TRY(last_launch());
+  route_scatter_kernel<<<nblk, 256, smem, s>>>(rt->T, rt->E, rt->k, rt->topk_ids, bc, rt->offsets, rt->row_offsets,
+                                               rt->sorted_to_slot, rt->slot_to_row);
+  return last_launch();
+}
+
+moesq_status route_launch(const float* logits, const moesq_routing* rt, int32_t* bc, cudaStream_t s) {
+  const int pl = (rt->E + 31) / 32;
+  if (pl <= 1) return route_launch_pl<1>(logits, rt, bc, s);
+  if (pl <= 2) return route_launch_pl<2>(logits, rt, bc, s);
+  if (pl <= 4) return route_launch_pl<4>(logits, rt, bc, s);
+  if (pl <= 8) return route_launch_pl<8>(logits, rt, bc, s);
+  if (pl <= 12) return route_launch_pl<12>(logits, rt, bc, s);
+  return route_launch_pl<16>(logits, rt, bc, s);
+}
+
 moesq_status check_layer(int T, int k, const moesq_weights* w_gu, const moesq_weights* w_dn) {
   MOESQ_TRY(check_weights(w_gu));
   MOESQ_TRY(check_weights(w_dn));
@@ -372,17 +404,7 @@ moesq_status moesq_route_permute(const float* logits, const moesq_routing* rt, v
   MOESQ_TRY(check_routing(rt));
   if (!logits) return MOESQ_ERR_INVALID_ARG;
   if (!workspace || workspace_bytes < moesq_route_workspace_bytes(rt->T, rt->E)) return MOESQ_ERR_WORKSPACE;
-  cudaStream_t s = as_stream(stream);
-  const int nblk = (rt->T + kRouteTPB - 1) / kRouteTPB;
-  int32_t* bc = static_cast<int32_t*>(workspace);
-  const size_t smem = (size_t)rt->E * kRouteWords * 4;
-  route_topk_kernel<<<nblk, 1024, smem, s>>>(logits, rt->T, rt->E, rt->k, rt->topk_ids, rt->topk_w, bc);
-  MOESQ_TRY(last_launch());
-  route_scan_kernel<<<1, 1024, 0, s>>>(bc, nblk, rt->E, rt->counts, rt->offsets, rt->row_offsets);
-  MOESQ_TRY(last_launch());
-  route_scatter_kernel<<<nblk, 256, smem, s>>>(rt->T, rt->E, rt->k, rt->topk_ids, bc, rt->offsets, rt->row_offsets,
-                                               rt->sorted_to_slot, rt->slot_to_row);
-  return last_launch();
+  return route_launch(logits, rt, static_cast<int32_t*>(workspace), as_stream(stream));
 }
 
 moesq_status moesq_quantize_act(const uint16_t* x_bf16, int T, int K, const moesq_routing* rt, const float* gamma,
@@ -405,7 +427,7 @@ moesq_status moesq_quantize_act(const uint16_t* x_bf16, int T, int K, const moes
     return MOESQ_ERR_INVALID_ARG;
   }
   cudaStream_t s = as_stream(stream);
-  const int64_t tasks = (int64_t)T * (rt ? k : 1) * (K / 256);
+  const int64_t tasks = (int64_t)T * (K / 256);
   quantize_act_kernel<<<grid_for(tasks, 8, device_info().sms), 256, 0, s>>>(x_bf16, T, K, k, ids, s2r, E, gamma,
                                                                             rows_cap, codes, scales);
   return last_launch();
@@ -454,7 +476,7 @@ moesq_status moesq_swiglu_quant(const uint16_t* y_gu, int I, const moesq_routing
   const int R = rt->T * rt->k;
   const int64_t tasks = (int64_t)R * (I / 256);
   swiglu_quant_kernel<<<grid_for(tasks, 8, device_info().sms), 256, 0, as_stream(stream)>>>(
-      y_gu, I, R, rt->E, rt->offsets, rt->row_offsets, gamma_h, h_codes, h_scales, nullptr);
+      y_gu, I, R, rt->E, rt->topk_ids, rt->slot_to_row, rt->rows_cap, gamma_h, h_codes, h_scales, nullptr);
   return last_launch();
 }
 
@@ -532,7 +554,7 @@ moesq_status moesq_calibrate_layer(const uint16_t* x_bf16, const float* logits, 
   MOESQ_CUDA(cudaMemsetAsync(gamma_a_dn, 0, sizeof(float) * E, s));
   const int R = T * k;
   swiglu_quant_kernel<<<grid_for((int64_t)R * (I / 256), 8, sms), 256, 0, s>>>(
-      ws.y_gu, I, R, E, rt.offsets, rt.row_offsets, nullptr, nullptr, nullptr,
+      ws.y_gu, I, R, E, rt.topk_ids, rt.slot_to_row, rt.rows_cap, nullptr, nullptr, nullptr,
       reinterpret_cast<unsigned int*>(gamma_a_dn));
   MOESQ_TRY(last_launch());
   amax_to_gamma_kernel<<<1, 1024, 0, s>>>(gamma_a_dn, E, 1);
@@ -552,17 +574,9 @@ moesq_status moesq_route_permute_noalloc(const float* logits, const moesq_routin
   if ((size_t)nblk * (size_t)rt->E > kNoAllocScratchInts) return MOESQ_ERR_UNSUPPORTED_SHAPE;
   int32_t* bc = route_scratch_device_ptr();
   if (!bc) return MOESQ_ERR_CUDA;
-  // route_topk_kernel writes every [block][expert] count the later kernels
+  // the counting kernel writes every [block][expert] count the later kernels
   // read, so the scratch needs no clearing between calls.
-  cudaStream_t s = as_stream(stream);
-  const size_t smem = (size_t)rt->E * kRouteWords * 4;
-  route_topk_kernel<<<nblk, 1024, smem, s>>>(logits, rt->T, rt->E, rt->k, rt->topk_ids, rt->topk_w, bc);
-  MOESQ_TRY(last_launch());
-  route_scan_kernel<<<1, 1024, 0, s>>>(bc, nblk, rt->E, rt->counts, rt->offsets, rt->row_offsets);
-  MOESQ_TRY(last_launch());
-  route_scatter_kernel<<<nblk, 256, smem, s>>>(rt->T, rt->E, rt->k, rt->topk_ids, bc, rt->offsets, rt->row_offsets,
-                                               rt->sorted_to_slot, rt->slot_to_row);
-  return last_launch();
+  return route_launch(logits, rt, bc, as_stream(stream));
 }
 
 }  // extern "C"

@@ -28,9 +28,11 @@ __device__ __forceinline__ void load8_bf16(const uint16_t* p, float (&v)[8]) {
   v[4] = bf16lo(u.z); v[5] = bf16hi(u.z); v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
 }
 
-// One warp task = (slot, 256-element chunk).  Dispatch form: slot (t, j)
-// writes token t quantised with gamma[topk_ids[slot]] to row slot_to_row[slot].
-// Plain form (slot_to_row == nullptr): slot t writes token t to row t with gamma[0].
+// One warp task = (token t, 256-element chunk).  The chunk of x[t] is read
+// once and the block amax computed once; it is then quantised for each of
+// the token's k slots with that slot's expert gamma and written to the
+// slot's row (the fused dispatch + quantisation).  Plain form
+// (slot_to_row == nullptr): k = 1, gamma[0], row = t.
 __global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t* __restrict__ x, int T, int K, int k,
                                                            const int32_t* __restrict__ topk_ids,
                                                            const int32_t* __restrict__ slot_to_row, int E,
@@ -38,50 +40,55 @@ __global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t* __res
                                                            uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
   const int lane = threadIdx.x & 31;
   const int chunks = K / 256;
-  const int64_t nslots = slot_to_row ? (int64_t)T * k : (int64_t)T;
-  const int64_t ntasks = nslots * chunks;
+  const int64_t ntasks = (int64_t)T * chunks;
   const int64_t wstride = (int64_t)gridDim.x * (blockDim.x >> 5);
   for (int64_t task = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); task < ntasks; task += wstride) {
-    const int64_t slot = task / chunks;
-    const int c = (int)(task % chunks);
-    int64_t t, row;
-    int e = 0;
+    const int64_t t = task / chunks;
+    const int c = (int)(task - t * chunks);
+    const int k0 = c * 256 + lane * 8;
+    // lane j < k holds slot j's row and gamma
+    int64_t my_row = t;
+    float my_gamma = 0.0f;
+    bool my_ok = true;
     if (slot_to_row) {
-      t = slot / k;
-      row = slot_to_row[slot];
-      e = topk_ids[slot];
-      if (e < 0 || e >= E || row < 0 || row >= rows_cap) {
+      if (lane < k) {
+        const int e = topk_ids[t * k + lane];
+        my_row = slot_to_row[t * k + lane];
+        my_ok = e >= 0 && e < E && my_row >= 0 && my_row < rows_cap;
+        my_gamma = my_ok ? gamma[e] : 0.0f;
+      }
+    } else if (lane == 0) {
+      my_gamma = gamma[0];
+    }
+    float v[8];
+    load8_bf16(x + t * K + k0, v);
+    float a = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(v[i]));
+    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+    const int nslots = slot_to_row ? k : 1;
+    for (int j = 0; j < nslots; ++j) {
+      const int64_t row = __shfl_sync(0xffffffffu, my_row, j);
+      const float g = __shfl_sync(0xffffffffu, my_gamma, j);
+      const bool ok = __shfl_sync(0xffffffffu, my_ok ? 1 : 0, j) != 0;
+      if (!ok) {
         if (lane == 0) record_error(kWhereQuant, kErrFault);
         continue;
       }
-    } else {
-      t = slot;
-      row = slot;
+      const uint32_t code = block_scale_code(g, a);
+      const uint32_t q = quant8(v, block_step(code, g), code == 0);
+      *reinterpret_cast<uint32_t*>(codes + row * (K / 2) + k0 / 2) = q;
+      if ((lane & 3) == 0) scales[mma_scale_offset(row, k0 / 32, K / 128)] = (uint8_t)code;
     }
-    const int k0 = c * 256 + lane * 8;
-    float v[8];
-    load8_bf16(x + t * K + k0, v);
-    uint32_t code;
-    const uint32_t q = quantize_lane8(v, gamma[e], &code);
-    *reinterpret_cast<uint32_t*>(codes + row * (K / 2) + k0 / 2) = q;
-    if ((lane & 3) == 0) scales[mma_scale_offset(row, k0 / 32, K / 128)] = (uint8_t)code;
   }
 }
 
-// Expert of compact position s: largest e with offsets[e] <= s.
-__device__ __forceinline__ int expert_of(const int32_t* __restrict__ offsets, int E, int s) {
-  int lo = 0, hi = E - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (offsets[mid] <= s) lo = mid; else hi = mid - 1;
-  }
-  return lo;
-}
-
-// SwiGLU + requantisation: one warp task = (compact row s, 256 outputs).
+// SwiGLU + requantisation: one warp task = (slot, 256 outputs); the slot's
+// expert and row come from the routing arrays.
 __global__ void __launch_bounds__(256) swiglu_quant_kernel(const uint16_t* __restrict__ y_gu, int I, int R, int E,
-                                                           const int32_t* __restrict__ offsets,
-                                                           const int32_t* __restrict__ row_offsets,
+                                                           const int32_t* __restrict__ topk_ids,
+                                                           const int32_t* __restrict__ slot_to_row, int rows_cap,
                                                            const float* __restrict__ gamma_h,
                                                            uint8_t* __restrict__ h_codes, uint8_t* __restrict__ h_scales,
                                                            unsigned int* __restrict__ amax_bits) {
@@ -90,10 +97,14 @@ __global__ void __launch_bounds__(256) swiglu_quant_kernel(const uint16_t* __res
   const int64_t ntasks = (int64_t)R * chunks;
   const int64_t wstride = (int64_t)gridDim.x * (blockDim.x >> 5);
   for (int64_t task = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); task < ntasks; task += wstride) {
-    const int s = (int)(task / chunks);
-    const int c = (int)(task % chunks);
-    const int e = expert_of(offsets, E, s);
-    const int64_t row = row_offsets[e] + (s - offsets[e]);
+    const int64_t slot = task / chunks;
+    const int c = (int)(task - slot * chunks);
+    const int e = topk_ids[slot];
+    const int64_t row = slot_to_row[slot];
+    if (e < 0 || e >= E || row < 0 || row >= rows_cap) {
+      if (lane == 0) record_error(kWhereSwiglu, kErrFault);
+      continue;
+    }
     const int i0 = c * 256 + lane * 8;
     float g[8], u[8], h[8];
     load8_bf16(y_gu + row * (2 * I) + i0, g);

@@ -25,67 +25,77 @@ __device__ __forceinline__ float from_ordered_bits(uint32_t o) {
   return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
 }
 
-// K1: one warp per token (32 warps, 4 tokens each, per 128-token block):
-// top-k by descending logit with ties to the lower id, softmax gate weights
-// over all E logits, and the block's per-expert token bitmaps -> per-block
-// counts [nblk][E].  Each pick is two warp reductions (max of the ordered
-// value, then min of the ids holding it).
-__global__ void __launch_bounds__(1024) route_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
-                                                          int32_t* __restrict__ topk_ids, float* __restrict__ topk_w,
+// Top-k of one token by one warp: PL logits per lane (lane + 32 i), softmax
+// over all E, k picks by descending logit with ties to the lower id.  Each
+// pick is two warp reductions (max of the ordered value, then min of the ids
+// holding it).  Lane (id % 32) of each pick writes ids / weights and, when
+// bitmap != nullptr, sets the token's bit (token index tl in its block).
+template <int PL>
+__device__ __forceinline__ void topk_one_token(const float* __restrict__ lr, int E, int k, int lane,
+                                               int32_t* __restrict__ ids_out, float* __restrict__ w_out,
+                                               uint32_t* bitmap, int tl) {
+  uint32_t o[PL];                        // ordered bits; the logit is recovered exactly from them
+  float mx = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < PL; ++i) {
+    const int e = lane + 32 * i;
+    const float x = (e < E) ? __ldg(lr + e) : -INFINITY;
+    o[i] = (e < E) ? ordered_bits(x) : 0u;
+    mx = fmaxf(mx, x);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  float z = 0.0f;
+#pragma unroll
+  for (int i = 0; i < PL; ++i)
+    if (lane + 32 * i < E) z += expf(from_ordered_bits(o[i]) - mx);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+  for (int j = 0; j < k; ++j) {
+    uint32_t bo = 0;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < PL; ++i)
+      if (o[i] > bo) { bo = o[i]; be = lane + 32 * i; }   // ids ascend with i: > keeps the lowest
+    const uint32_t best = __reduce_max_sync(0xffffffffu, bo);
+    const int win = __reduce_min_sync(0xffffffffu, (bo == best && be < E) ? be : 0x7fffffff);
+    if (win >= E) {                      // only NaN logits leave no candidate
+      if (lane == 0) record_error(kWhereRoute, kErrFault);
+      return;
+    }
+    if ((win & 31) == lane) {
+#pragma unroll
+      for (int i = 0; i < PL; ++i)
+        if (i == (win >> 5)) o[i] = 0u;  // taken
+      ids_out[j] = win;
+      w_out[j] = __fdiv_rn(expf(from_ordered_bits(best) - mx), z);
+      if (bitmap) atomicOr(&bitmap[win * kRouteWords + (tl >> 5)], 1u << (tl & 31));
+    }
+  }
+}
+
+// K1: one warp per token over the whole grid: ids and gate weights.
+template <int PL>
+__global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                         int32_t* __restrict__ topk_ids, float* __restrict__ topk_w) {
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  topk_one_token<PL>(logits + (size_t)t * E, E, k, threadIdx.x & 31, topk_ids + (size_t)t * k,
+                     topk_w + (size_t)t * k, nullptr, 0);
+}
+
+// K1b: per 128-token block, per-expert counts from the block's token bitmaps.
+__global__ void __launch_bounds__(256) route_count_kernel(int T, int E, int k, const int32_t* __restrict__ topk_ids,
                                                           int32_t* __restrict__ block_counts) {
   extern __shared__ uint32_t bitmap[];                 // [E][kRouteWords]
   for (int i = threadIdx.x; i < E * kRouteWords; i += blockDim.x) bitmap[i] = 0;
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-  const int per_lane = (E + 31) >> 5;
-  for (int tl = warp; tl < kRouteTPB; tl += nwarps) {
-    const int t = blockIdx.x * kRouteTPB + tl;
-    if (t >= T) break;
-    const float* lr = logits + (size_t)t * E;
-    uint32_t o[kRouteMaxPerLane];          // ordered bits; the logit is recovered exactly from them
-    float mx = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < kRouteMaxPerLane; ++i) {
-      const int e = lane + 32 * i;
-      const float x = (i < per_lane && e < E) ? __ldg(lr + e) : -INFINITY;
-      o[i] = (i < per_lane && e < E) ? ordered_bits(x) : 0u;
-      mx = fmaxf(mx, x);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    float z = 0.0f;
-#pragma unroll
-    for (int i = 0; i < kRouteMaxPerLane; ++i) {
-      const int e = lane + 32 * i;
-      if (i < per_lane && e < E) z += expf(from_ordered_bits(o[i]) - mx);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
-    uint32_t taken = 0;
-    for (int j = 0; j < k; ++j) {
-      uint32_t bo = 0;
-      int be = 0x7fffffff;
-#pragma unroll
-      for (int i = 0; i < kRouteMaxPerLane; ++i) {
-        const int e = lane + 32 * i;
-        if (i < per_lane && e < E && !(taken >> i & 1u) && o[i] > bo) {   // ids ascend with i: > keeps the lowest
-          bo = o[i];
-          be = e;
-        }
-      }
-      const uint32_t best = __reduce_max_sync(0xffffffffu, bo);
-      const int win = __reduce_min_sync(0xffffffffu, (bo == best && be < E) ? be : 0x7fffffff);
-      if (win >= E) {                      // only NaN logits leave no candidate
-        if (lane == 0) record_error(kWhereRoute, kErrFault);
-        break;
-      }
-      if ((win & 31) == lane) {
-        taken |= 1u << (win >> 5);
-        topk_ids[(size_t)t * k + j] = win;
-        topk_w[(size_t)t * k + j] = __fdiv_rn(expf(from_ordered_bits(bo) - mx), z);
-        atomicOr(&bitmap[win * kRouteWords + (tl >> 5)], 1u << (tl & 31));
-      }
-    }
+  const int t0 = blockIdx.x * kRouteTPB;
+  const int nslots = min(kRouteTPB, T - t0) * k;
+  for (int i = threadIdx.x; i < nslots; i += blockDim.x) {
+    const int tl = i / k;
+    const int e = topk_ids[(size_t)t0 * k + i];
+    if (e >= 0 && e < E) atomicOr(&bitmap[e * kRouteWords + (tl >> 5)], 1u << (tl & 31));
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -184,6 +194,81 @@ __global__ void __launch_bounds__(256) route_scatter_kernel(int T, int E, int k,
     const int local = block_base[(size_t)blockIdx.x * E + e] + rank;
     sorted_to_slot[offsets[e] + local] = slot;
     slot_to_row[slot] = row_offsets[e] + local;
+  }
+}
+
+// Single-CTA routing for T <= kRouteTPB (one token block): top-k, counts,
+// offsets and the scatter in one launch, with the same arithmetic as the
+// three-kernel path (K1 body, K2's scan, K3's ranks).
+template <int PL>
+__global__ void __launch_bounds__(1024) route_small_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                           int32_t* __restrict__ topk_ids, float* __restrict__ topk_w,
+                                                           int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                                                           int32_t* __restrict__ row_offsets,
+                                                           int32_t* __restrict__ sorted_to_slot,
+                                                           int32_t* __restrict__ slot_to_row) {
+  extern __shared__ uint32_t bitmap[];                 // [E][kRouteWords]
+  __shared__ int32_t s_cnt[kRouteMaxE];
+  __shared__ int32_t s_off[kRouteMaxE];
+  __shared__ int32_t s_roff[kRouteMaxE];
+  for (int i = threadIdx.x; i < E * kRouteWords; i += blockDim.x) bitmap[i] = 0;
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  for (int tl = warp; tl < T; tl += nwarps)
+    topk_one_token<PL>(logits + (size_t)tl * E, E, k, lane, topk_ids + (size_t)tl * k, topk_w + (size_t)tl * k,
+                       bitmap, tl);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int c = 0;
+#pragma unroll
+    for (int w = 0; w < kRouteWords; ++w) c += __popc(bitmap[e * kRouteWords + w]);
+    s_cnt[e] = c;
+    counts[e] = c;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int per = (E + 31) / 32, e0 = lane * per;
+    int sc = 0, sr = 0;
+    for (int i = 0; i < per; ++i) {
+      const int e = e0 + i;
+      if (e < E) { sc += s_cnt[e]; sr += (s_cnt[e] + 127) & ~127; }
+    }
+    int ic = sc, ir = sr;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int tc = __shfl_up_sync(0xffffffffu, ic, off);
+      const int tr = __shfl_up_sync(0xffffffffu, ir, off);
+      if (lane >= off) { ic += tc; ir += tr; }
+    }
+    int oc = ic - sc, orr = ir - sr;
+    for (int i = 0; i < per; ++i) {
+      const int e = e0 + i;
+      if (e < E) {
+        s_off[e] = oc;
+        s_roff[e] = orr;
+        offsets[e] = oc;
+        row_offsets[e] = orr;
+        oc += s_cnt[e];
+        orr += (s_cnt[e] + 127) & ~127;
+      }
+    }
+    if (lane == 31) { offsets[E] = ic; row_offsets[E] = ir; }
+  }
+  __syncthreads();
+  const int nslots = T * k;
+  for (int i = threadIdx.x; i < nslots; i += blockDim.x) {
+    const int tl = i / k;
+    const int e = topk_ids[i];
+    if (e < 0 || e >= E) continue;
+    int rank = 0;
+#pragma unroll
+    for (int w = 0; w < kRouteWords; ++w) {
+      const uint32_t word = bitmap[e * kRouteWords + w];
+      if (w < (tl >> 5)) rank += __popc(word);
+      else if (w == (tl >> 5)) rank += __popc(word & ((1u << (tl & 31)) - 1u));
+    }
+    sorted_to_slot[s_off[e] + rank] = i;
+    slot_to_row[i] = s_roff[e] + rank;
   }
 }
 
