@@ -14,13 +14,16 @@
 //           pre-swizzled compressed values, 2 KB of metadata, 1 KB of scales);
 //           TMA brings the token codes (TN x 128 B, 128-byte swizzle) and a bulk
 //           copy their scales (1 KB) into an S-stage shared-memory ring.
-//   warp 1  MMA issuer (one thread): tcgen05.cp moves metadata and both scale
-//           blocks from shared memory into tensor memory, then two
+//   warp 2  copy issuer (one thread): tcgen05.cp moves the stage's metadata
+//           and both scale blocks into one of 4 rotating TMEM buffers.
+//   warp 1  MMA issuer (one thread): two
 //           tcgen05.mma.sp.kind::mxf4nvf4.block_scale (K = 128 dense each)
-//           accumulate in TMEM; tcgen05.commit frees the stage.  Accumulators
-//           are double-buffered in TMEM so the epilogue of tile i overlaps
-//           the main loop of tile i+1.
-//   warps 2-5 epilogue: tcgen05.ld of the fp32 accumulator, times alpha_e,
+//           per K step accumulate in TMEM; tcgen05.commit frees the stage and
+//           the TMEM buffer.  Issuing copies and MMAs from two threads lets
+//           the two run side by side (one thread issuing both serialises
+//           them).  Accumulators are double-buffered in TMEM so the epilogue
+//           of tile i overlaps the main loop of tile i+1.
+//   warps 3-6 epilogue: tcgen05.ld of the fp32 accumulator, times alpha_e,
 //           rounded to bf16 and stored for the valid rows only.
 // Work units are (expert, 128-row weight block, TN-row token block); the
 // per-expert token counts stay on the device and every CTA derives the unit
@@ -35,7 +38,8 @@
 namespace moesq {
 
 constexpr int kGemmMaxE = 512;
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 224;   // producer, MMA, copy, 4 epilogue warps
+constexpr int kTmemBufs = 4;        // rotating TMEM buffers of metadata + scales
 
 template <int TN>
 struct GemmCfg {
@@ -47,18 +51,20 @@ struct GemmCfg {
   static constexpr int kOffB = kOffW + kStages * kWBytes;
   static constexpr int kOffSfb = kOffB + kStages * kBBytes;
   static constexpr int kOffBar = kOffSfb + kStages * kSfBytes;
-  static constexpr int kNumBars = 2 * kStages + 5;  // full, empty, acc_full[2], acc_empty[2], drain
+  // full[S], empty[S], acc_full[2], acc_empty[2], drain, tready[kTmemBufs], tfree[kTmemBufs]
+  static constexpr int kNumBars = 2 * kStages + 5 + 2 * kTmemBufs;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kOffTab = kOffMisc + 16;
   static constexpr int kSmemBytes = kOffTab + (3 * kGemmMaxE + 1) * 4 + 1024;
   static constexpr uint32_t kTmemCols = (TN == 128) ? 512 : 256;
-  static constexpr uint32_t kColE = 2 * TN;
-  static constexpr uint32_t kColSfa = 2 * TN + 4;
-  static constexpr uint32_t kColSfb = 2 * TN + 12;
+  // TMEM buffer b (of kTmemBufs) at column kColBuf + 20 b: metadata 4 columns,
+  // weight scales 8, token scales 8
+  static constexpr uint32_t kColBuf = 2 * TN;
+  static constexpr uint32_t kBufCols = 20;
   static_assert(TN == 64 || TN == 128, "token tile");
   static_assert(kWBytes % 1024 == 0 && kBBytes % 1024 == 0, "1 KB aligned stages");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
-  static_assert(kColSfb + 8 <= kTmemCols, "tensor memory");
+  static_assert(kColBuf + kTmemBufs * kBufCols <= kTmemCols, "tensor memory");
 };
 
 struct GemmParams {
@@ -122,12 +128,15 @@ grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const GemmP
   auto accf_bar = [&](int b) { return bar(2 * C::kStages + b); };
   auto acce_bar = [&](int b) { return bar(2 * C::kStages + 2 + b); };
   const uint32_t drain_bar = bar(2 * C::kStages + 4);
+  auto tready_bar = [&](int b) { return bar(2 * C::kStages + 5 + b); };
+  auto tfree_bar = [&](int b) { return bar(2 * C::kStages + 5 + kTmemBufs + b); };
 
   // ---------------------------------------------------------------- set-up
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
     for (int b = 0; b < 2; ++b) { mbar_init(accf_bar(b), 1); mbar_init(acce_bar(b), 4); }
     mbar_init(drain_bar, 1);
+    for (int b = 0; b < kTmemBufs; ++b) { mbar_init(tready_bar(b), 1); mbar_init(tfree_bar(b), 1); }
     fence_barrier_init();
     misc[1] = 0;
     prefetch_tmap(&tm_b);
@@ -218,9 +227,13 @@ grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const GemmP
       }
     }
   } else if (warp == 1) {
+    // MMA issuer: per K step waits for the stage (A / B in shared memory)
+    // and for its TMEM buffer of metadata + scales, issues the two sparse
+    // MMAs, then frees both.
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      uint32_t g = 0;                   // K steps of this CTA so far (TMEM buffer = g % kTmemBufs)
       bool ok = true, any = false;
       int it = 0;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
@@ -236,8 +249,11 @@ grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const GemmP
         tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(buf * TN);
         const uint32_t idesc = idesc_sp_nvf4((uint32_t)tl.nmma);
-        for (int kt = 0; kt < KT; ++kt) {
-          if (!mbar_wait(full_bar(stage), phase, p.timeout_ns, abort_flag)) {
+        for (int kt = 0; kt < KT; ++kt, ++g) {
+          const int tb = (int)(g % kTmemBufs);
+          const uint32_t tph = (g / kTmemBufs) & 1u;
+          if (!mbar_wait(full_bar(stage), phase, p.timeout_ns, abort_flag) ||
+              !mbar_wait(tready_bar(tb), tph, p.timeout_ns, abort_flag)) {
             record_error(kWhereGemmMma, kErrTimeout);
             *abort_flag = 1;
             ok = false;
@@ -246,23 +262,17 @@ grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const GemmP
           tc_fence_after();
           const uint32_t sa = sbase + C::kOffW + stage * C::kWBytes;
           const uint32_t sb = sbase + C::kOffB + stage * C::kBBytes;
-          const uint32_t se = sa + kKTileMeta;
-          const uint32_t ssa = sa + kKTileScales;
-          const uint32_t ssb = sbase + C::kOffSfb + stage * C::kSfBytes;
-          tc_cp_128x128b(tmem + C::kColE, smem_desc(se, 16, 128, 0));
-          tc_cp_32x128b_x4(tmem + C::kColSfa, smem_desc(ssa, 16, 128, 0));
-          tc_cp_32x128b_x4(tmem + C::kColSfa + 4, smem_desc(ssa + 512, 16, 128, 0));
-          tc_cp_32x128b_x4(tmem + C::kColSfb, smem_desc(ssb, 16, 128, 0));
-          tc_cp_32x128b_x4(tmem + C::kColSfb + 4, smem_desc(ssb + 512, 16, 128, 0));
+          const uint32_t tbuf = tmem + C::kColBuf + C::kBufCols * (uint32_t)tb;
 #pragma unroll
           for (int kb = 0; kb < 2; ++kb) {
             const uint64_t adesc = smem_desc(sa + kb * 32, 16, 512, 4);     // 64-byte swizzle
             const uint64_t bdesc = smem_desc(sb + kb * 64, 16, 1024, 2);    // 128-byte swizzle
-            tc_mma_sp_nvf4(d_tmem, adesc, bdesc, tmem + C::kColE + 2 * kb, idesc, tmem + C::kColSfa + 4 * kb,
-                           tmem + C::kColSfb + 4 * kb + tl.q, (kt | kb) != 0 ? 1u : 0u);
+            tc_mma_sp_nvf4(d_tmem, adesc, bdesc, tbuf + 2 * kb, idesc, tbuf + 4 + 4 * kb,
+                           tbuf + 12 + 4 * kb + tl.q, (kt | kb) != 0 ? 1u : 0u);
           }
           any = true;
           tc_commit(empty_bar(stage));
+          tc_commit(tfree_bar(tb));
           if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
         }
         if (ok) tc_commit(accf_bar(buf));
@@ -273,8 +283,48 @@ grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const GemmP
         mbar_wait(drain_bar, 0, p.timeout_ns, &zero);
       }
     }
+  } else if (warp == 2) {
+    // Copy issuer: per K step moves the stage's metadata and both scale blocks
+    // from shared memory into a free TMEM buffer (tcgen05.cp), so that these
+    // copies run alongside the MMAs of earlier steps.
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t g = 0;
+      bool ok = true, any = false;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        for (int kt = 0; kt < KT; ++kt, ++g) {
+          const int tb = (int)(g % kTmemBufs);
+          const uint32_t tph = (g / kTmemBufs) & 1u;
+          if (!mbar_wait(full_bar(stage), phase, p.timeout_ns, abort_flag) ||
+              !mbar_wait(tfree_bar(tb), tph ^ 1u, p.timeout_ns, abort_flag)) {
+            record_error(kWhereGemmMma, kErrTimeout);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = sbase + C::kOffW + stage * C::kWBytes;
+          const uint32_t ssb = sbase + C::kOffSfb + stage * C::kSfBytes;
+          const uint32_t tbuf = tmem + C::kColBuf + C::kBufCols * (uint32_t)tb;
+          tc_cp_128x128b(tbuf, smem_desc(sa + kKTileMeta, 16, 128, 0));
+          tc_cp_32x128b_x4(tbuf + 4, smem_desc(sa + kKTileScales, 16, 128, 0));
+          tc_cp_32x128b_x4(tbuf + 8, smem_desc(sa + kKTileScales + 512, 16, 128, 0));
+          tc_cp_32x128b_x4(tbuf + 12, smem_desc(ssb, 16, 128, 0));
+          tc_cp_32x128b_x4(tbuf + 16, smem_desc(ssb + 512, 16, 128, 0));
+          any = true;
+          tc_commit(tready_bar(tb));
+          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok && any) {                 // let the copies in flight land before TMEM is released
+        int zero = 0;
+        tc_commit(drain_bar);
+        mbar_wait(drain_bar, 0, p.timeout_ns, &zero);
+      }
+    }
   } else {
-    const int quad = warp & 3;          // TMEM lanes 32*quad .. 32*quad+31
+    const int quad = warp & 3;          // warps 3..6: TMEM lanes 32*quad .. 32*quad+31
     int it = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
       const Tile tl = decode_tile<TN>(t, MB, E, ntp, rstart, cnt);
