@@ -23,6 +23,8 @@ inputs and output in pinned host memory (copies inside the timed region).
 from __future__ import annotations
 
 import argparse
+import glob
+import hashlib
 import json
 import os
 import statistics
@@ -60,12 +62,41 @@ WORKLOADS = {
 DEFAULT_WORKLOAD = "30b_layer_t256"
 
 
+FP4_OVER_BF16 = 4.0    # nominal dense tensor-core ratio, fp4 : bf16 (9 : 2.25 PFLOP/s)
+SPARSE_FACTOR = 2.0    # a structured-sparse MMA runs the dense-equivalent contraction at twice the rate
+
+
 def load_peaks():
+    """HBM copy GB/s and dense bf16 TFLOP/s (burst) measured on this GPU type,
+    else an earlier measurement of the same pool."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
-        return d.get("hbm_gbs", 6650.0), "measured"
-    return 6650.0, "fallback"
+        return {"hbm_gbs": d.get("hbm_gbs", 6650.0), "bf16_tflops": d.get("bf16_tflops", 1590.0),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+def gemm_source_sha():
+    """Hash of the sources the grouped GEMM kernel is built from; a DRAM
+    traffic record taken with ncu is only used while it matches."""
+    h = hashlib.sha256()
+    for f in ("gemm.cuh", "common.cuh"):
+        h.update(open(os.path.join(ROOT, "grouped_gemm_moesq_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload, gemm):
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum)
+    from the ncu summaries under profiles/, or None."""
+    sha = gemm_source_sha()
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        for ln in open(path):
+            if ln.startswith("traffic-record: "):
+                rec = json.loads(ln[len("traffic-record: "):])
+                if rec.get("workload") == workload and rec.get("gemm") == gemm and rec.get("source_sha") == sha:
+                    return rec["dram_bytes_per_launch"]
+    return None
 
 
 # ------------------------------------------------------------------ clocks
@@ -117,21 +148,24 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ work accounting
 def step_work(E, k, H, I, T, counts_gu, kind):
-    """(flops, weight bytes, per-GEMM algorithmic bytes) of one step."""
+    """(flops, weight bytes, per-GEMM algorithmic bytes, per-GEMM dense-equivalent
+    flops) of one step."""
     R = T * k
     touched = int((np.asarray(counts_gu) > 0).sum())
     if kind == "gemm_down":
         M, K = H, I
         flops = 2.0 * M * K * R
         wbytes = touched * packed_weight_bytes(M, K)
-        return flops, wbytes, {"down": wbytes + R * (K // 2 + K // 32) + R * M * 2}
+        return flops, wbytes, {"down": wbytes + R * (K // 2 + K // 32) + R * M * 2}, {"down": flops}
     gu_w = touched * packed_weight_bytes(2 * I, H)
     gu_bytes = gu_w + R * (H // 2 + H // 32) + R * 2 * I * 2
+    gu_fl = 2.0 * 2 * I * H * R
     if kind == "gemm":
-        return 2.0 * 2 * I * H * R, gu_w, {"gate_up": gu_bytes}
+        return gu_fl, gu_w, {"gate_up": gu_bytes}, {"gate_up": gu_fl}
     dn_w = touched * packed_weight_bytes(H, I)
     dn_bytes = dn_w + R * (I // 2 + I // 32) + R * H * 2
-    return 2.0 * (2 * I * H + H * I) * R, gu_w + dn_w, {"gate_up": gu_bytes, "down": dn_bytes}
+    dn_fl = 2.0 * H * I * R
+    return gu_fl + dn_fl, gu_w + dn_w, {"gate_up": gu_bytes, "down": dn_bytes}, {"gate_up": gu_fl, "down": dn_fl}
 
 
 def logits_for(routing, seed, T, E):
@@ -214,7 +248,8 @@ def run_cuda(args, rank, world, local_rank):
         for _, f in comps:
             f()
 
-    launches_per_step = 8 if kind == "layer" else 5
+    # routing: one fused kernel for T <= 128 tokens, else top-k, count, scan and scatter
+    launches_per_step = (1 if T <= 128 else 4) + 2 + (3 if kind == "layer" else 0)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
         flush.zero_()
@@ -313,7 +348,7 @@ def run_cuda(args, rank, world, local_rank):
         e2e = {"ms_per_step": statistics.mean(e2e_ms),
                "h2d_bytes_per_step": T * H * 2 + T * E * 4, "d2h_bytes_per_step": T * H * 2}
 
-    flops, wbytes, gemm_bytes = step_work(E, k, H, I, T, counts, kind)
+    flops, wbytes, gemm_bytes, gemm_fl = step_work(E, k, H, I, T, counts, kind)
     t_max = ms
     if world > 1:
         tt = torch.tensor([ms, e2e["ms_per_step"] if e2e else 0.0], device=dev)
@@ -322,7 +357,7 @@ def run_cuda(args, rank, world, local_rank):
         if e2e:
             e2e["ms_per_step"] = float(tt[1])
     return dict(kind=kind, E=E, k=k, H=H, I=I, T=T, routing=routing, ms=t_max, parts=parts, flops=flops,
-                wbytes=wbytes, gemm_bytes=gemm_bytes, e2e=e2e, clocks=clk, launches=launches_per_step * args.steps,
+                wbytes=wbytes, gemm_bytes=gemm_bytes, gemm_fl=gemm_fl, e2e=e2e, clocks=clk, launches=launches_per_step * args.steps,
                 wall_s=t_wall, counts=counts)
 
 
@@ -437,18 +472,31 @@ def main():
             dist.destroy_process_group()
         return
 
-    hbm_peak, peak_kind = load_peaks()
+    peaks = load_peaks()
     ms = r["ms"]
     value = world * r["flops"] / (ms * 1e-3) / 1e12
     weight_gbs = world * r["wbytes"] / (ms * 1e-3) / 1e9
-    gemm_key = "gemm_main"
-    gemm_ms = r["parts"][gemm_key]
-    gbytes = r["gemm_bytes"]["down" if r["kind"] == "gemm_down" else "gate_up"]
-    achieved = gbytes / (gemm_ms * 1e-3) / 1e9
-    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved / hbm_peak, "traffic": None,
-                "kernel": "grouped_sparse_gemm (%s)" % ("down" if r["kind"] == "gemm_down" else "gate_up"),
-                "kernel_ms": gemm_ms, "peak_source": peak_kind}
+    gname = "down" if r["kind"] == "gemm_down" else "gate_up"
+    gemm_ms = r["parts"]["gemm_main"]
+    gbytes, gfl = r["gemm_bytes"][gname], r["gemm_fl"][gname]
+    # the bound is whichever ideal time is longer: algorithmic bytes at the HBM
+    # copy rate, or dense-equivalent flops at the sparse NVFP4 tensor rate
+    hbm_peak = peaks["hbm_gbs"]
+    tc_peak = peaks["bf16_tflops"] * FP4_OVER_BF16 * SPARSE_FACTOR
+    hbm_ach = gbytes / (gemm_ms * 1e-3) / 1e9
+    tc_ach = gfl / (gemm_ms * 1e-3) / 1e12
+    traffic = profiled_traffic(args.workload, gname)
+    if gbytes / (hbm_peak * 1e9) >= gfl / (tc_peak * 1e12):
+        roofline = {"bound": "hbm", "achieved": hbm_ach, "peak": hbm_peak, "unit": "GB/s",
+                    "frac": hbm_ach / hbm_peak}
+    else:
+        roofline = {"bound": "tensor", "achieved": tc_ach, "peak": tc_peak, "unit": "TFLOP/s",
+                    "frac": tc_ach / tc_peak}
+    roofline.update({"traffic": traffic, "algorithmic_bytes": gbytes, "dense_equiv_flops": gfl,
+                     "kernel": "grouped_sparse_gemm (%s)" % gname, "kernel_ms": gemm_ms,
+                     "hbm_frac": hbm_ach / hbm_peak, "tensor_frac": tc_ach / tc_peak,
+                     "peak_source": "%s (tensor peak = dense bf16 burst x %g fp4/bf16 x %g sparse)"
+                     % (peaks["source"], FP4_OVER_BF16, SPARSE_FACTOR)})
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "nvfp4 (e2m1 x ue4m3 products, f32 accumulate, bf16 out)",
