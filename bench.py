@@ -168,6 +168,29 @@ def step_work(E, k, H, I, T, counts_gu, kind):
     return gu_fl + dn_fl, gu_w + dn_w, {"gate_up": gu_bytes, "down": dn_bytes}, {"gate_up": gu_fl, "down": dn_fl}
 
 
+def rank_seed(seed, rank):
+    """Seed of one rank's token batch: every rank draws its own batch
+    (independent replicas, weak scaling)."""
+    return seed + 7919 * rank
+
+
+def max_over_ranks(values, device="cpu"):
+    """Element-wise maximum of a list of floats over all ranks of the default
+    process group (identity without one).  Every rank must call it."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def job_throughput(flops_per_rank, world, ms):
+    """Whole-job TFLOP/s: all ranks' work over the slowest rank's time."""
+    return world * flops_per_rank / (ms * 1e-3) / 1e12
+
+
 def logits_for(routing, seed, T, E):
     return S.zipf_logits_np(seed, T, E) if routing == "zipf" else S.uniform_logits_np(seed, T, E)
 
@@ -207,8 +230,8 @@ def run_cuda(args, rank, world, local_rank):
 
     # per-rank batch (independent replicas: weak scaling, no data-path collective)
     K_in = I if kind == "gemm_down" else H
-    x_np = S.activations_bf16_np(seed + 7919 * rank, T, K_in)
-    lg_np = logits_for(routing, seed + 7919 * rank, T, E)
+    x_np = S.activations_bf16_np(rank_seed(seed, rank), T, K_in)
+    lg_np = logits_for(routing, rank_seed(seed, rank), T, E)
     x = torch.from_numpy(x_np.view(np.int16).copy()).to(dev).view(torch.bfloat16)
     lg = torch.from_numpy(lg_np).to(dev)
 
@@ -349,13 +372,9 @@ def run_cuda(args, rank, world, local_rank):
                "h2d_bytes_per_step": T * H * 2 + T * E * 4, "d2h_bytes_per_step": T * H * 2}
 
     flops, wbytes, gemm_bytes, gemm_fl = step_work(E, k, H, I, T, counts, kind)
-    t_max = ms
-    if world > 1:
-        tt = torch.tensor([ms, e2e["ms_per_step"] if e2e else 0.0], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_max = float(tt[0])
-        if e2e:
-            e2e["ms_per_step"] = float(tt[1])
+    t_max, e2e_max = max_over_ranks([ms, e2e["ms_per_step"] if e2e else 0.0], device=dev)
+    if e2e:
+        e2e["ms_per_step"] = e2e_max
     return dict(kind=kind, E=E, k=k, H=H, I=I, T=T, routing=routing, ms=t_max, parts=parts, flops=flops,
                 wbytes=wbytes, gemm_bytes=gemm_bytes, gemm_fl=gemm_fl, e2e=e2e, clocks=clk, launches=launches_per_step * args.steps,
                 wall_s=t_wall, counts=counts)
@@ -474,7 +493,7 @@ def main():
 
     peaks = load_peaks()
     ms = r["ms"]
-    value = world * r["flops"] / (ms * 1e-3) / 1e12
+    value = job_throughput(r["flops"], world, ms)
     weight_gbs = world * r["wbytes"] / (ms * 1e-3) / 1e9
     gname = "down" if r["kind"] == "gemm_down" else "gate_up"
     gemm_ms = r["parts"]["gemm_main"]
@@ -507,7 +526,7 @@ def main():
                             "touched": int((r["counts"] > 0).sum())}}
     if r["e2e"]:
         e = r["e2e"]
-        line["e2e"] = {"value": world * r["flops"] / (e["ms_per_step"] * 1e-3) / 1e12, "unit": "TFLOP/s",
+        line["e2e"] = {"value": job_throughput(r["flops"], world, e["ms_per_step"]), "unit": "TFLOP/s",
                        "h2d_bytes_per_step": e["h2d_bytes_per_step"], "d2h_bytes_per_step": e["d2h_bytes_per_step"],
                        "ms_per_step": e["ms_per_step"]}
     if world == 1 and not args.no_cpu_baseline:

@@ -1,0 +1,64 @@
+"""Multi-rank host logic of bench.py on CPU: two gloo ranks, as torchrun
+would launch them on two GPUs.  Each rank draws its own token batch (weak
+scaling, no data-path collective); the only collective is the max of the
+timings over ranks, and the job throughput counts every rank's work over the
+slowest rank's time."""
+import json
+import os
+import socket
+
+import numpy as np
+import pytest
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, out_dir):
+    import datetime
+
+    import torch.distributed as dist
+
+    import bench
+    import synthetic as S
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        ms = [1.0 + rank, 5.0 - rank, 0.25 * rank]          # rank 1 is slower in the first entry only
+        got = bench.max_over_ranks(ms)
+        x = S.activations_bf16_np(bench.rank_seed(1234, rank), 4, 64)
+        lg = bench.logits_for("zipf", bench.rank_seed(1234, rank), 4, 16)
+        dist.barrier()
+        with open(os.path.join(out_dir, "rank%d.json" % rank), "w") as f:
+            json.dump({"max": got, "x": x.astype(np.int64).tolist(), "lg": lg.tolist()}, f)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_max_and_own_batches(tmp_path):
+    mp = pytest.importorskip("torch.multiprocessing")
+    world = 2
+    mp.spawn(_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True)
+    r = [json.load(open(tmp_path / ("rank%d.json" % i))) for i in range(world)]
+    for i in range(world):
+        assert r[i]["max"] == [2.0, 5.0, 0.25]
+    assert r[0]["x"] != r[1]["x"]                            # independent token batches
+    assert r[0]["lg"] != r[1]["lg"]
+
+
+def test_single_process_max_is_identity():
+    import bench
+    assert bench.max_over_ranks([3.0, 0.5]) == [3.0, 0.5]
+
+
+def test_job_throughput_counts_all_ranks_over_slowest():
+    import bench
+    # 4 ranks, 1e12 dense-equivalent flops each, slowest rank 2 ms
+    assert bench.job_throughput(1e12, 4, 2.0) == pytest.approx(2000.0)
+    assert bench.rank_seed(7, 0) == 7 and bench.rank_seed(7, 3) != bench.rank_seed(7, 2)
