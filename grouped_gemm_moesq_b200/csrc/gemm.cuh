@@ -8,7 +8,7 @@
 // the expert are operand B (N <= TN per tile), both block scales are applied
 // inside the MMA and alpha_e in the epilogue (App. D.1).
 //
-// Design (one CTA per SM, persistent, warp-specialised):
+// Design (two CTAs per SM, persistent, warp-specialised):
 //   warp 0  producer: per 256-wide K step one bulk copy brings the weight
 //           tile of the kernel form (11 KB, contiguous: 128 x 64 B of
 //           pre-swizzled compressed values, 2 KB of metadata, 1 KB of scales);
@@ -21,8 +21,10 @@
 //           per K step accumulate in TMEM; tcgen05.commit frees the stage and
 //           the TMEM buffer.  Issuing copies and MMAs from two threads lets
 //           the two run side by side (one thread issuing both serialises
-//           them).  Accumulators are double-buffered in TMEM so the epilogue
-//           of tile i overlaps the main loop of tile i+1.
+//           them).  With 64-row token tiles the accumulator is
+//           double-buffered in TMEM so the epilogue of tile i overlaps the
+//           main loop of tile i+1; with 128-row tiles the other CTA of the SM
+//           keeps the tensor pipe busy during an epilogue.
 //   warps 3-6 epilogue: tcgen05.ld of the fp32 accumulator, times alpha_e,
 //           rounded to bf16 and stored for the valid rows only.
 // Work units are (expert, 128-row weight block, TN-row token block); the
@@ -39,11 +41,15 @@ namespace moesq {
 
 constexpr int kGemmMaxE = 512;
 constexpr int kGemmThreads = 224;   // producer, MMA, copy, 4 epilogue warps
-constexpr int kTmemBufs = 4;        // rotating TMEM buffers of metadata + scales
 
 template <int TN>
 struct GemmCfg {
-  static constexpr int kStages = (TN == 128) ? 7 : 10;
+  // Two CTAs share an SM: each is one copy -> MMA issue chain, and two
+  // independent chains keep the tensor pipe busier than one (a chain waits,
+  // per K step, for its copies to land before its MMAs can go).
+  static constexpr int kCtasPerSm = 2;
+  static constexpr int kNAcc = (TN == 128) ? 1 : 2;     // accumulator buffers (TN columns each)
+  static constexpr int kStages = (TN == 128) ? 3 : 5;
   static constexpr int kWBytes = kKTileBytes;    // weight tile: A image, metadata, scales
   static constexpr int kBBytes = TN * 128;       // token codes, 256 K
   static constexpr int kSfBytes = 1024;          // token scales: 2 x (32 x 16 B)
@@ -51,20 +57,21 @@ struct GemmCfg {
   static constexpr int kOffB = kOffW + kStages * kWBytes;
   static constexpr int kOffSfb = kOffB + kStages * kBBytes;
   static constexpr int kOffBar = kOffSfb + kStages * kSfBytes;
-  // full[S], empty[S], acc_full[2], acc_empty[2], drain, tready[kTmemBufs], tfree[kTmemBufs]
-  static constexpr int kNumBars = 2 * kStages + 5 + 2 * kTmemBufs;
+  static constexpr int kTBufs = 4;                       // rotating TMEM buffers of metadata + scales
+  // full[S], empty[S], acc_full[2], acc_empty[2], drain, tready[kTBufs], tfree[kTBufs]
+  static constexpr int kNumBars = 2 * kStages + 5 + 2 * kTBufs;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kOffTab = kOffMisc + 16;
   static constexpr int kSmemBytes = kOffTab + (3 * kGemmMaxE + 1) * 4 + 1024;
-  static constexpr uint32_t kTmemCols = (TN == 128) ? 512 : 256;
-  // TMEM buffer b (of kTmemBufs) at column kColBuf + 20 b: metadata 4 columns,
+  static constexpr uint32_t kTmemCols = 256;            // half of an SM's tensor memory
+  // TMEM buffer b (of kTBufs) at column kColBuf + 20 b: metadata 4 columns,
   // weight scales 8, token scales 8
-  static constexpr uint32_t kColBuf = 2 * TN;
+  static constexpr uint32_t kColBuf = kNAcc * TN;
   static constexpr uint32_t kBufCols = 20;
   static_assert(TN == 64 || TN == 128, "token tile");
   static_assert(kWBytes % 1024 == 0 && kBBytes % 1024 == 0, "1 KB aligned stages");
-  static_assert(kSmemBytes <= 227 * 1024, "shared memory");
-  static_assert(kColBuf + kTmemBufs * kBufCols <= kTmemCols, "tensor memory");
+  static_assert(kCtasPerSm * (kSmemBytes + 1024) <= 228 * 1024, "shared memory of the CTAs of one SM");
+  static_assert(kColBuf + kTBufs * kBufCols <= kTmemCols, "tensor memory");
 };
 
 struct GemmParams {
@@ -108,7 +115,7 @@ __device__ __forceinline__ Tile decode_tile(int t, int MB, int E, const int* ntp
 }
 
 template <int TN>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(kGemmThreads, GemmCfg<TN>::kCtasPerSm)
 grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const GemmParams p) {
   using C = GemmCfg<TN>;
   extern __shared__ uint8_t smem_raw[];
@@ -129,14 +136,14 @@ grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const GemmP
   auto acce_bar = [&](int b) { return bar(2 * C::kStages + 2 + b); };
   const uint32_t drain_bar = bar(2 * C::kStages + 4);
   auto tready_bar = [&](int b) { return bar(2 * C::kStages + 5 + b); };
-  auto tfree_bar = [&](int b) { return bar(2 * C::kStages + 5 + kTmemBufs + b); };
+  auto tfree_bar = [&](int b) { return bar(2 * C::kStages + 5 + C::kTBufs + b); };
 
   // ---------------------------------------------------------------- set-up
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
     for (int b = 0; b < 2; ++b) { mbar_init(accf_bar(b), 1); mbar_init(acce_bar(b), 4); }
     mbar_init(drain_bar, 1);
-    for (int b = 0; b < kTmemBufs; ++b) { mbar_init(tready_bar(b), 1); mbar_init(tfree_bar(b), 1); }
+    for (int b = 0; b < C::kTBufs; ++b) { mbar_init(tready_bar(b), 1); mbar_init(tfree_bar(b), 1); }
     fence_barrier_init();
     misc[1] = 0;
     prefetch_tmap(&tm_b);
@@ -233,13 +240,13 @@ grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const GemmP
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t g = 0;                   // K steps of this CTA so far (TMEM buffer = g % kTmemBufs)
+      uint32_t g = 0;                   // K steps of this CTA so far (TMEM buffer = g % kTBufs)
       bool ok = true, any = false;
       int it = 0;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
         const Tile tl = decode_tile<TN>(t, MB, E, ntp, rstart, cnt);
-        const int buf = it & 1;
-        const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+        const int buf = it % C::kNAcc;
+        const uint32_t aph = (uint32_t)(it / C::kNAcc) & 1u;
         if (!mbar_wait(acce_bar(buf), aph ^ 1u, p.timeout_ns, abort_flag)) {
           record_error(kWhereGemmMma, kErrTimeout);
           *abort_flag = 1;
@@ -250,8 +257,8 @@ grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const GemmP
         const uint32_t d_tmem = tmem + (uint32_t)(buf * TN);
         const uint32_t idesc = idesc_sp_nvf4((uint32_t)tl.nmma);
         for (int kt = 0; kt < KT; ++kt, ++g) {
-          const int tb = (int)(g % kTmemBufs);
-          const uint32_t tph = (g / kTmemBufs) & 1u;
+          const int tb = (int)(g % C::kTBufs);
+          const uint32_t tph = (g / C::kTBufs) & 1u;
           if (!mbar_wait(full_bar(stage), phase, p.timeout_ns, abort_flag) ||
               !mbar_wait(tready_bar(tb), tph, p.timeout_ns, abort_flag)) {
             record_error(kWhereGemmMma, kErrTimeout);
@@ -294,8 +301,8 @@ grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const GemmP
       bool ok = true, any = false;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
         for (int kt = 0; kt < KT; ++kt, ++g) {
-          const int tb = (int)(g % kTmemBufs);
-          const uint32_t tph = (g / kTmemBufs) & 1u;
+          const int tb = (int)(g % C::kTBufs);
+          const uint32_t tph = (g / C::kTBufs) & 1u;
           if (!mbar_wait(full_bar(stage), phase, p.timeout_ns, abort_flag) ||
               !mbar_wait(tfree_bar(tb), tph ^ 1u, p.timeout_ns, abort_flag)) {
             record_error(kWhereGemmMma, kErrTimeout);
@@ -328,8 +335,8 @@ grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const GemmP
     int it = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
       const Tile tl = decode_tile<TN>(t, MB, E, ntp, rstart, cnt);
-      const int buf = it & 1;
-      const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+      const int buf = it % C::kNAcc;
+      const uint32_t aph = (uint32_t)(it / C::kNAcc) & 1u;
       if (!mbar_wait(accf_bar(buf), aph, p.timeout_ns, abort_flag)) {
         if (lane == 0) { record_error(kWhereGemmEpilogue, kErrTimeout); *abort_flag = 1; }
         break;

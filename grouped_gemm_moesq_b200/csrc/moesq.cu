@@ -152,7 +152,7 @@ moesq_status launch_gemm(const moesq_weights* w, const uint8_t* a_codes, const u
   p.K = w->K;
   p.rows_cap = rows_cap;
   p.timeout_ns = g_timeout_ns;
-  const int grid = num_ctas > 0 ? num_ctas : di.sms;
+  const int grid = num_ctas > 0 ? num_ctas : di.sms * C::kCtasPerSm;
   grouped_sparse_gemm_kernel<TN><<<grid, kGemmThreads, C::kSmemBytes, s>>>(tmb, p);
   return last_launch();
 }
