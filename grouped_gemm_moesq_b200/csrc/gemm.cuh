@@ -196,7 +196,7 @@ grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const GemmP
   // ---------------------------------------------------------------- roles
   if (warp == 0) {
     if (lane == 0) {
-      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_w = policy_evict_last();
       const uint64_t pol_x = policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
