@@ -14,18 +14,19 @@
 //           pre-swizzled compressed values, 2 KB of metadata, 1 KB of scales);
 //           TMA brings the token codes (TN x 128 B, 128-byte swizzle) and a bulk
 //           copy their scales (1 KB) into an S-stage shared-memory ring.
-//   warp 2  copy issuer (one thread): tcgen05.cp moves the stage's metadata
-//           and both scale blocks into one of 4 rotating TMEM buffers.
-//   warp 1  MMA issuer (one thread): two
-//           tcgen05.mma.sp.kind::mxf4nvf4.block_scale (K = 128 dense each)
-//           per K step accumulate in TMEM; tcgen05.commit frees the stage and
-//           the TMEM buffer.  Issuing copies and MMAs from two threads lets
-//           the two run side by side (one thread issuing both serialises
-//           them).  With 64-row token tiles the accumulator is
-//           double-buffered in TMEM so the epilogue of tile i overlaps the
-//           main loop of tile i+1; with 128-row tiles the other CTA of the SM
-//           keeps the tensor pipe busy during an epilogue.
-//   warps 3-6 epilogue: tcgen05.ld of the fp32 accumulator, times alpha_e,
+//   warp 1  MMA issuer (one thread): per K step tcgen05.cp moves the
+//           metadata and both scale blocks into one of 4 rotating TMEM
+//           buffers, then two tcgen05.mma.sp.kind::mxf4nvf4.block_scale
+//           (K = 128 dense each) accumulate in TMEM; tcgen05.commit frees the
+//           stage.  A thread's copies and MMAs execute in issue order, so
+//           they need no barrier between them; handing the copies to another
+//           warp costs a commit/wait round trip per K step and measured
+//           slower.  The second CTA of the SM is a second independent issue
+//           stream, which keeps the tensor pipe busy.  With 64-row token tiles
+//           the accumulator is double-buffered in TMEM so the epilogue of tile
+//           i overlaps the main loop of tile i+1; with 128-row tiles the other
+//           CTA covers the epilogue.
+//   warps 2-5 epilogue: tcgen05.ld of the fp32 accumulator, times alpha_e,
 //           rounded to bf16 and stored for the valid rows only.
 // Work units are (expert, 128-row weight block, TN-row token block); the
 // per-expert token counts stay on the device and every CTA derives the unit
@@ -40,7 +41,7 @@
 namespace moesq {
 
 constexpr int kGemmMaxE = 512;
-constexpr int kGemmThreads = 224;   // producer, MMA, copy, 4 epilogue warps
+constexpr int kGemmThreads = 192;   // producer, MMA, 4 epilogue warps
 
 template <int TN>
 struct GemmCfg {
@@ -58,8 +59,8 @@ struct GemmCfg {
   static constexpr int kOffSfb = kOffB + kStages * kBBytes;
   static constexpr int kOffBar = kOffSfb + kStages * kSfBytes;
   static constexpr int kTBufs = 4;                       // rotating TMEM buffers of metadata + scales
-  // full[S], empty[S], acc_full[2], acc_empty[2], drain, tready[kTBufs], tfree[kTBufs]
-  static constexpr int kNumBars = 2 * kStages + 5 + 2 * kTBufs;
+  // full[S], empty[S], acc_full[2], acc_empty[2], drain
+  static constexpr int kNumBars = 2 * kStages + 5;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kOffTab = kOffMisc + 16;
   static constexpr int kSmemBytes = kOffTab + (3 * kGemmMaxE + 1) * 4 + 1024;
@@ -135,15 +136,12 @@ grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const GemmP
   auto accf_bar = [&](int b) { return bar(2 * C::kStages + b); };
   auto acce_bar = [&](int b) { return bar(2 * C::kStages + 2 + b); };
   const uint32_t drain_bar = bar(2 * C::kStages + 4);
-  auto tready_bar = [&](int b) { return bar(2 * C::kStages + 5 + b); };
-  auto tfree_bar = [&](int b) { return bar(2 * C::kStages + 5 + C::kTBufs + b); };
 
   // ---------------------------------------------------------------- set-up
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) { mbar_init(full_bar(s), 1); mbar_init(empty_bar(s), 1); }
     for (int b = 0; b < 2; ++b) { mbar_init(accf_bar(b), 1); mbar_init(acce_bar(b), 4); }
     mbar_init(drain_bar, 1);
-    for (int b = 0; b < C::kTBufs; ++b) { mbar_init(tready_bar(b), 1); mbar_init(tfree_bar(b), 1); }
     fence_barrier_init();
     misc[1] = 0;
     prefetch_tmap(&tm_b);
@@ -196,7 +194,11 @@ grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const GemmP
   // ---------------------------------------------------------------- roles
   if (warp == 0) {
     if (lane == 0) {
-      const uint64_t pol_w = policy_evict_last();
+      // weight tiles an expert reuses (more than one token block) stay in
+      // L2; tiles read once are streamed with evict_first so they do not
+      // push out the token tiles
+      const uint64_t pol_keep = policy_evict_last();
+      const uint64_t pol_stream = policy_evict_first();
       const uint64_t pol_x = policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
@@ -207,6 +209,7 @@ grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const GemmP
         const int nbox = (tl.nmma + 31) >> 5;
         const uint32_t bytes = C::kWBytes + C::kSfBytes + nbox * 4096;
         const uint8_t* wt = p.ktiles + ((int64_t)tl.e * MB + tl.mb) * KT * C::kWBytes;
+        const uint64_t pol_w = (ntp[tl.e + 1] - ntp[tl.e] > 1) ? pol_keep : pol_stream;
         const uint8_t* xsc = p.a_scales + (int64_t)(tl.row0 >> 7) * KB * 512;
         for (int kt = 0; kt < KT; ++kt) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, p.timeout_ns, abort_flag)) {
@@ -234,9 +237,12 @@ grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const GemmP
       }
     }
   } else if (warp == 1) {
-    // MMA issuer: per K step waits for the stage (A / B in shared memory)
-    // and for its TMEM buffer of metadata + scales, issues the two sparse
-    // MMAs, then frees both.
+    // MMA issuer: per K step waits for the stage, moves its metadata and
+    // both scale blocks into the next of kTBufs rotating TMEM buffers
+    // (tcgen05.cp) and issues the two sparse MMAs that read them.  The
+    // copies and MMAs of one thread run in issue order, so no barrier
+    // separates them; the buffer rotation keeps a copy away from the
+    // buffers the MMAs in flight still read.
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
@@ -258,9 +264,7 @@ grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const GemmP
         const uint32_t idesc = idesc_sp_nvf4((uint32_t)tl.nmma);
         for (int kt = 0; kt < KT; ++kt, ++g) {
           const int tb = (int)(g % C::kTBufs);
-          const uint32_t tph = (g / C::kTBufs) & 1u;
-          if (!mbar_wait(full_bar(stage), phase, p.timeout_ns, abort_flag) ||
-              !mbar_wait(tready_bar(tb), tph, p.timeout_ns, abort_flag)) {
+          if (!mbar_wait(full_bar(stage), phase, p.timeout_ns, abort_flag)) {
             record_error(kWhereGemmMma, kErrTimeout);
             *abort_flag = 1;
             ok = false;
@@ -269,7 +273,13 @@ grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const GemmP
           tc_fence_after();
           const uint32_t sa = sbase + C::kOffW + stage * C::kWBytes;
           const uint32_t sb = sbase + C::kOffB + stage * C::kBBytes;
+          const uint32_t ssb = sbase + C::kOffSfb + stage * C::kSfBytes;
           const uint32_t tbuf = tmem + C::kColBuf + C::kBufCols * (uint32_t)tb;
+          tc_cp_128x128b(tbuf, smem_desc(sa + kKTileMeta, 16, 128, 0));
+          tc_cp_32x128b_x4(tbuf + 4, smem_desc(sa + kKTileScales, 16, 128, 0));
+          tc_cp_32x128b_x4(tbuf + 8, smem_desc(sa + kKTileScales + 512, 16, 128, 0));
+          tc_cp_32x128b_x4(tbuf + 12, smem_desc(ssb, 16, 128, 0));
+          tc_cp_32x128b_x4(tbuf + 16, smem_desc(ssb + 512, 16, 128, 0));
 #pragma unroll
           for (int kb = 0; kb < 2; ++kb) {
             const uint64_t adesc = smem_desc(sa + kb * 32, 16, 512, 4);     // 64-byte swizzle
@@ -279,7 +289,6 @@ grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const GemmP
           }
           any = true;
           tc_commit(empty_bar(stage));
-          tc_commit(tfree_bar(tb));
           if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
         }
         if (ok) tc_commit(accf_bar(buf));
@@ -290,48 +299,8 @@ grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const GemmP
         mbar_wait(drain_bar, 0, p.timeout_ns, &zero);
       }
     }
-  } else if (warp == 2) {
-    // Copy issuer: per K step moves the stage's metadata and both scale blocks
-    // from shared memory into a free TMEM buffer (tcgen05.cp), so that these
-    // copies run alongside the MMAs of earlier steps.
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t g = 0;
-      bool ok = true, any = false;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        for (int kt = 0; kt < KT; ++kt, ++g) {
-          const int tb = (int)(g % C::kTBufs);
-          const uint32_t tph = (g / C::kTBufs) & 1u;
-          if (!mbar_wait(full_bar(stage), phase, p.timeout_ns, abort_flag) ||
-              !mbar_wait(tfree_bar(tb), tph ^ 1u, p.timeout_ns, abort_flag)) {
-            record_error(kWhereGemmMma, kErrTimeout);
-            *abort_flag = 1;
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t sa = sbase + C::kOffW + stage * C::kWBytes;
-          const uint32_t ssb = sbase + C::kOffSfb + stage * C::kSfBytes;
-          const uint32_t tbuf = tmem + C::kColBuf + C::kBufCols * (uint32_t)tb;
-          tc_cp_128x128b(tbuf, smem_desc(sa + kKTileMeta, 16, 128, 0));
-          tc_cp_32x128b_x4(tbuf + 4, smem_desc(sa + kKTileScales, 16, 128, 0));
-          tc_cp_32x128b_x4(tbuf + 8, smem_desc(sa + kKTileScales + 512, 16, 128, 0));
-          tc_cp_32x128b_x4(tbuf + 12, smem_desc(ssb, 16, 128, 0));
-          tc_cp_32x128b_x4(tbuf + 16, smem_desc(ssb + 512, 16, 128, 0));
-          any = true;
-          tc_commit(tready_bar(tb));
-          if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
-        }
-      }
-      if (!ok && any) {                 // let the copies in flight land before TMEM is released
-        int zero = 0;
-        tc_commit(drain_bar);
-        mbar_wait(drain_bar, 0, p.timeout_ns, &zero);
-      }
-    }
   } else {
-    const int quad = warp & 3;          // warps 3..6: TMEM lanes 32*quad .. 32*quad+31
+    const int quad = warp & 3;          // warps 2..5: TMEM lanes 32*quad .. 32*quad+31
     int it = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
       const Tile tl = decode_tile<TN>(t, MB, E, ntp, rstart, cnt);

@@ -228,9 +228,11 @@ template <int PL>
 moesq_status route_launch_pl(const float* logits, const moesq_routing* rt, int32_t* bc, cudaStream_t s) {
   const int nblk = (rt->T + kRouteTPB - 1) / kRouteTPB;
   const size_t smem = (size_t)rt->E * kRouteWords * 4;
-  if (nblk == 1) {                      // one token block: fused single-CTA path
-    route_small_kernel<PL><<<1, 1024, smem, s>>>(logits, rt->T, rt->E, rt->k, rt->topk_ids, rt->topk_w, rt->counts,
-                                                 rt->offsets, rt->row_offsets, rt->sorted_to_slot, rt->slot_to_row);
+  if (rt->T <= kRouteSmallMaxT) {       // few tokens: fused single-CTA path
+    const int words = (rt->T + 31) / 32;
+    route_small_kernel<PL><<<1, 1024, (size_t)rt->E * words * 4, s>>>(
+        logits, rt->T, rt->E, rt->k, rt->topk_ids, rt->topk_w, rt->counts, rt->offsets, rt->row_offsets,
+        rt->sorted_to_slot, rt->slot_to_row, words);
     return last_launch();
   }
   route_topk_kernel<PL><<<(rt->T + 7) / 8, 256, 0, s>>>(logits, rt->T, rt->E, rt->k, rt->topk_ids, rt->topk_w);

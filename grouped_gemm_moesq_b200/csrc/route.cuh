@@ -10,6 +10,7 @@ namespace moesq {
 
 constexpr int kRouteTPB = 128;          // tokens per routing block
 constexpr int kRouteWords = kRouteTPB / 32;
+constexpr int kRouteSmallMaxT = 128;     // tokens routed by the single-CTA kernel
 constexpr int kRouteMaxE = 512;
 constexpr int kRouteMaxPerLane = kRouteMaxE / 32;
 
@@ -29,11 +30,12 @@ __device__ __forceinline__ float from_ordered_bits(uint32_t o) {
 // over all E, k picks by descending logit with ties to the lower id.  Each
 // pick is two warp reductions (max of the ordered value, then min of the ids
 // holding it).  Lane (id % 32) of each pick writes ids / weights and, when
-// bitmap != nullptr, sets the token's bit (token index tl in its block).
+// bitmap != nullptr, sets the token's bit (token index tl in its block; the
+// bitmap holds `words` 32-bit words per expert).
 template <int PL>
 __device__ __forceinline__ void topk_one_token(const float* __restrict__ lr, int E, int k, int lane,
                                                int32_t* __restrict__ ids_out, float* __restrict__ w_out,
-                                               uint32_t* bitmap, int tl) {
+                                               uint32_t* bitmap, int words, int tl) {
   uint32_t o[PL];                        // ordered bits; the logit is recovered exactly from them
   float mx = -INFINITY;
 #pragma unroll
@@ -69,7 +71,7 @@ __device__ __forceinline__ void topk_one_token(const float* __restrict__ lr, int
         if (i == (win >> 5)) o[i] = 0u;  // taken
       ids_out[j] = win;
       w_out[j] = __fdiv_rn(expf(from_ordered_bits(best) - mx), z);
-      if (bitmap) atomicOr(&bitmap[win * kRouteWords + (tl >> 5)], 1u << (tl & 31));
+      if (bitmap) atomicOr(&bitmap[win * words + (tl >> 5)], 1u << (tl & 31));
     }
   }
 }
@@ -81,7 +83,7 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
   topk_one_token<PL>(logits + (size_t)t * E, E, k, threadIdx.x & 31, topk_ids + (size_t)t * k,
-                     topk_w + (size_t)t * k, nullptr, 0);
+                     topk_w + (size_t)t * k, nullptr, 0, 0);
 }
 
 // K1b: per 128-token block, per-expert counts from the block's token bitmaps.
@@ -197,31 +199,30 @@ __global__ void __launch_bounds__(256) route_scatter_kernel(int T, int E, int k,
   }
 }
 
-// Single-CTA routing for T <= kRouteTPB (one token block): top-k, counts,
-// offsets and the scatter in one launch, with the same arithmetic as the
-// three-kernel path (K1 body, K2's scan, K3's ranks).
+// Single-CTA routing for T <= kRouteSmallMaxT tokens: top-k, counts, offsets
+// and the scatter in one launch, with the same arithmetic as the multi-kernel
+// path; the expert bitmaps hold words = ceil(T / 32) words each.
 template <int PL>
 __global__ void __launch_bounds__(1024) route_small_kernel(const float* __restrict__ logits, int T, int E, int k,
                                                            int32_t* __restrict__ topk_ids, float* __restrict__ topk_w,
                                                            int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                                                            int32_t* __restrict__ row_offsets,
                                                            int32_t* __restrict__ sorted_to_slot,
-                                                           int32_t* __restrict__ slot_to_row) {
-  extern __shared__ uint32_t bitmap[];                 // [E][kRouteWords]
+                                                           int32_t* __restrict__ slot_to_row, int words) {
+  extern __shared__ uint32_t bitmap[];                 // [E][words]
   __shared__ int32_t s_cnt[kRouteMaxE];
   __shared__ int32_t s_off[kRouteMaxE];
   __shared__ int32_t s_roff[kRouteMaxE];
-  for (int i = threadIdx.x; i < E * kRouteWords; i += blockDim.x) bitmap[i] = 0;
+  for (int i = threadIdx.x; i < E * words; i += blockDim.x) bitmap[i] = 0;
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
   for (int tl = warp; tl < T; tl += nwarps)
     topk_one_token<PL>(logits + (size_t)tl * E, E, k, lane, topk_ids + (size_t)tl * k, topk_w + (size_t)tl * k,
-                       bitmap, tl);
+                       bitmap, words, tl);
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int c = 0;
-#pragma unroll
-    for (int w = 0; w < kRouteWords; ++w) c += __popc(bitmap[e * kRouteWords + w]);
+    for (int w = 0; w < words; ++w) c += __popc(bitmap[e * words + w]);
     s_cnt[e] = c;
     counts[e] = c;
   }
@@ -261,12 +262,8 @@ __global__ void __launch_bounds__(1024) route_small_kernel(const float* __restri
     const int e = topk_ids[i];
     if (e < 0 || e >= E) continue;
     int rank = 0;
-#pragma unroll
-    for (int w = 0; w < kRouteWords; ++w) {
-      const uint32_t word = bitmap[e * kRouteWords + w];
-      if (w < (tl >> 5)) rank += __popc(word);
-      else if (w == (tl >> 5)) rank += __popc(word & ((1u << (tl & 31)) - 1u));
-    }
+    for (int w = 0; w < (tl >> 5); ++w) rank += __popc(bitmap[e * words + w]);
+    rank += __popc(bitmap[e * words + (tl >> 5)] & ((1u << (tl & 31)) - 1u));
     sorted_to_slot[s_off[e] + rank] = i;
     slot_to_row[i] = s_roff[e] + rank;
   }
