@@ -97,13 +97,55 @@ __device__ __forceinline__ uint32_t block_scale_code(float gamma, float amax_b) 
 __device__ __forceinline__ float block_step(uint32_t code, float gamma) {
   return __fdiv_rn(ue4m3_value(code), gamma);
 }
-// Eight values of one block -> four bytes of codes (x / s_b onto E2M1).
-__device__ __forceinline__ uint32_t quant8(const float (&v)[8], float s_b, bool zero_block) {
-  if (zero_block) return 0u;
+// Eight values of one block -> four bytes of codes: each code is the E2M1
+// rounding of the correctly rounded quotient q = fl(v / s_b), given
+// r = fl(1 / s_b) (rfin: r is finite).
+//
+// The code of q only depends on where q lies relative to the E2M1 decision
+// points (0.25, 0.75, ..., 5) and on exact ties there, and E2M1 rounding is
+// monotone in the magnitude.  y = fl(v * r) is within (2^-23 + 2^-48)|x| of
+// x = v / s_b, and q within 2^-24 |x| of x, so q lies strictly inside
+// [y (1 - 2^-20), y (1 + 2^-20)] (both ends rounded).  When the two ends
+// round to the same codes, every value between them does, q included, and
+// those codes are returned.  Otherwise (a value within about 2^-20 of a
+// decision point), or when r is not finite, the quotients are formed exactly.
+__device__ __forceinline__ uint32_t quant8_r(const float* v, float s_b, float r, bool rfin) {
+  if (rfin) {
+    float lo[8], hi[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float y = __fmul_rn(v[i], r);
+      lo[i] = __fmul_rn(y, 0x1.ffffep-1f);     // 1 - 2^-20
+      hi[i] = __fmul_rn(y, 0x1.00001p+0f);     // 1 + 2^-20
+    }
+    const uint32_t cl = e2m1x8(lo), ch = e2m1x8(hi);
+    if (cl == ch) return cl;
+  }
   float q[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) q[i] = __fdiv_rn(v[i], s_b);
   return e2m1x8(q);
+}
+
+// Eight values of one block -> four bytes of codes (x / s_b onto E2M1).
+__device__ __forceinline__ uint32_t quant8(const float (&v)[8], float s_b, bool zero_block) {
+  if (zero_block) return 0u;
+  const float r = __frcp_rn(s_b);
+  return quant8_r(v, s_b, r, isfinite(r));
+}
+
+// One whole 32-element scale block -> 16 bytes of codes (element 2i in the
+// low nibble of byte i).
+__device__ __forceinline__ uint4 quant32(const float (&v)[32], float s_b, bool zero_block) {
+  if (zero_block) return make_uint4(0u, 0u, 0u, 0u);
+  const float r = __frcp_rn(s_b);
+  const bool rfin = isfinite(r);
+  uint4 o;
+  o.x = quant8_r(v, s_b, r, rfin);
+  o.y = quant8_r(v + 8, s_b, r, rfin);
+  o.z = quant8_r(v + 16, s_b, r, rfin);
+  o.w = quant8_r(v + 24, s_b, r, rfin);
+  return o;
 }
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }

@@ -413,7 +413,7 @@ moesq_status moesq_quantize_act(const uint16_t* x_bf16, int T, int K, const moes
                                 int rows_cap, uint8_t* codes, uint8_t* scales, void* stream) {
   if (!x_bf16 || !gamma || !codes || !scales) return MOESQ_ERR_INVALID_ARG;
   if (T < 1 || K < 256 || K % 256) return MOESQ_ERR_UNSUPPORTED_SHAPE;
-  if (!aligned(x_bf16, 16) || !aligned(codes, 4)) return MOESQ_ERR_INVALID_ARG;
+  if (!aligned(x_bf16, 16) || !aligned(codes, 16)) return MOESQ_ERR_INVALID_ARG;
   if (rows_cap < 128 || rows_cap % 128) return MOESQ_ERR_INVALID_ARG;
   int k = 1, E = 1;
   const int32_t* ids = nullptr;
@@ -429,7 +429,7 @@ moesq_status moesq_quantize_act(const uint16_t* x_bf16, int T, int K, const moes
     return MOESQ_ERR_INVALID_ARG;
   }
   cudaStream_t s = as_stream(stream);
-  const int64_t tasks = (int64_t)T * (K / 256);
+  const int64_t tasks = (int64_t)T * k * ((K + 1023) / 1024);
   quantize_act_kernel<<<grid_for(tasks, 8, device_info().sms), 256, 0, s>>>(x_bf16, T, K, k, ids, s2r, E, gamma,
                                                                             rows_cap, codes, scales);
   return last_launch();
@@ -475,8 +475,9 @@ moesq_status moesq_swiglu_quant(const uint16_t* y_gu, int I, const moesq_routing
   MOESQ_TRY(check_routing(rt));
   if (!y_gu || !gamma_h || !h_codes || !h_scales) return MOESQ_ERR_INVALID_ARG;
   if (I < 256 || I % 256) return MOESQ_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(y_gu, 16) || !aligned(h_codes, 16)) return MOESQ_ERR_INVALID_ARG;
   const int R = rt->T * rt->k;
-  const int64_t tasks = (int64_t)R * (I / 256);
+  const int64_t tasks = (int64_t)R * ((I + 1023) / 1024);
   swiglu_quant_kernel<<<grid_for(tasks, 8, device_info().sms), 256, 0, as_stream(stream)>>>(
       y_gu, I, R, rt->E, rt->topk_ids, rt->slot_to_row, rt->rows_cap, gamma_h, h_codes, h_scales, nullptr);
   return last_launch();
@@ -555,7 +556,7 @@ moesq_status moesq_calibrate_layer(const uint16_t* x_bf16, const float* logits, 
                                       gamma_a_gu, ws.y_gu, nullptr, s));
   MOESQ_CUDA(cudaMemsetAsync(gamma_a_dn, 0, sizeof(float) * E, s));
   const int R = T * k;
-  swiglu_quant_kernel<<<grid_for((int64_t)R * (I / 256), 8, sms), 256, 0, s>>>(
+  swiglu_quant_kernel<<<grid_for((int64_t)R * ((I + 1023) / 1024), 8, sms), 256, 0, s>>>(
       ws.y_gu, I, R, E, rt.topk_ids, rt.slot_to_row, rt.rows_cap, nullptr, nullptr, nullptr,
       reinterpret_cast<unsigned int*>(gamma_a_dn));
   MOESQ_TRY(last_launch());

@@ -1,26 +1,13 @@
 // Activation-side kernels: NVFP4 quantisation of activations (plain and
 // fused with the dispatch scatter), SwiGLU + requantisation, the
 // router-weighted combine and the amax reductions behind the static global
-// scales.  All are HBM / L2 bound: one warp streams 256 contiguous elements
-// (16-byte loads per lane, 4 lanes per 32-element scale block).
+// scales.  The quantising kernels give each lane one whole 32-element scale
+// block (64-byte loads, one scale per lane, 16-byte code stores), so the
+// block's scale and step are computed once.
 #pragma once
 #include "common.cuh"
 
 namespace moesq {
-
-// Quantises 8 values held by this lane; the 4 lanes of a 32-element block
-// share amax through shuffles.  Returns the 4 code bytes; *code_out gets the
-// block's scale code.
-__device__ __forceinline__ uint32_t quantize_lane8(const float (&v)[8], float gamma, uint32_t* code_out) {
-  float a = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(v[i]));
-  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
-  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
-  const uint32_t code = block_scale_code(gamma, a);
-  *code_out = code;
-  return quant8(v, block_step(code, gamma), code == 0);
-}
 
 __device__ __forceinline__ void load8_bf16(const uint16_t* p, float (&v)[8]) {
   const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
@@ -28,64 +15,72 @@ __device__ __forceinline__ void load8_bf16(const uint16_t* p, float (&v)[8]) {
   v[4] = bf16lo(u.z); v[5] = bf16hi(u.z); v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
 }
 
-// One warp task = (token t, 256-element chunk).  The chunk of x[t] is read
-// once and the block amax computed once; it is then quantised for each of
-// the token's k slots with that slot's expert gamma and written to the
-// slot's row (the fused dispatch + quantisation).  Plain form
-// (slot_to_row == nullptr): k = 1, gamma[0], row = t.
+__device__ __forceinline__ void load32_bf16(const uint16_t* p, float (&v)[32]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p) + j);
+    v[8 * j + 0] = bf16lo(u.x); v[8 * j + 1] = bf16hi(u.x); v[8 * j + 2] = bf16lo(u.y); v[8 * j + 3] = bf16hi(u.y);
+    v[8 * j + 4] = bf16lo(u.z); v[8 * j + 5] = bf16hi(u.z); v[8 * j + 6] = bf16lo(u.w); v[8 * j + 7] = bf16hi(u.w);
+  }
+}
+
+// Quantises the 32-element block v with global scale gamma: stores the 16
+// code bytes at dst and returns the block's scale code.
+__device__ __forceinline__ uint32_t quantize_block32(const float (&v)[32], float gamma, uint8_t* dst) {
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) a = fmaxf(a, fabsf(v[i]));
+  const uint32_t code = block_scale_code(gamma, a);
+  *reinterpret_cast<uint4*>(dst) = quant32(v, block_step(code, gamma), code == 0);
+  return code;
+}
+
+// One warp task = (slot, 1024-element chunk of the slot's token): lane l
+// quantises the scale block [1024 c + 32 l, +32) of x[t] with the slot's
+// expert gamma into the slot's row (the fused dispatch + quantisation).
+// Consecutive tasks walk the chunks, then the k slots of a token, so the
+// token's row is re-read from L2.  Plain form (slot_to_row == nullptr): one
+// slot per token, gamma[0], row = t.
 __global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t* __restrict__ x, int T, int K, int k,
                                                            const int32_t* __restrict__ topk_ids,
                                                            const int32_t* __restrict__ slot_to_row, int E,
                                                            const float* __restrict__ gamma, int rows_cap,
                                                            uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
   const int lane = threadIdx.x & 31;
-  const int chunks = K / 256;
-  const int64_t ntasks = (int64_t)T * chunks;
+  const int chunks = (K + 1023) / 1024;
+  const int nslots = slot_to_row ? k : 1;
+  const int64_t ntasks = (int64_t)T * nslots * chunks;
   const int64_t wstride = (int64_t)gridDim.x * (blockDim.x >> 5);
   for (int64_t task = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); task < ntasks; task += wstride) {
-    const int64_t t = task / chunks;
-    const int c = (int)(task - t * chunks);
-    const int k0 = c * 256 + lane * 8;
-    // lane j < k holds slot j's row and gamma
-    int64_t my_row = t;
-    float my_gamma = 0.0f;
-    bool my_ok = true;
+    const int64_t slot = task / chunks;
+    const int c = (int)(task - slot * chunks);
+    const int64_t t = slot / nslots;
+    int64_t row = t;
+    float g;
     if (slot_to_row) {
-      if (lane < k) {
-        const int e = topk_ids[t * k + lane];
-        my_row = slot_to_row[t * k + lane];
-        my_ok = e >= 0 && e < E && my_row >= 0 && my_row < rows_cap;
-        my_gamma = my_ok ? gamma[e] : 0.0f;
-      }
-    } else if (lane == 0) {
-      my_gamma = gamma[0];
-    }
-    float v[8];
-    load8_bf16(x + t * K + k0, v);
-    float a = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(v[i]));
-    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
-    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
-    const int nslots = slot_to_row ? k : 1;
-    for (int j = 0; j < nslots; ++j) {
-      const int64_t row = __shfl_sync(0xffffffffu, my_row, j);
-      const float g = __shfl_sync(0xffffffffu, my_gamma, j);
-      const bool ok = __shfl_sync(0xffffffffu, my_ok ? 1 : 0, j) != 0;
-      if (!ok) {
+      const int e = topk_ids[slot];
+      row = slot_to_row[slot];
+      if (e < 0 || e >= E || row < 0 || row >= rows_cap) {
         if (lane == 0) record_error(kWhereQuant, kErrFault);
         continue;
       }
-      const uint32_t code = block_scale_code(g, a);
-      const uint32_t q = quant8(v, block_step(code, g), code == 0);
-      *reinterpret_cast<uint32_t*>(codes + row * (K / 2) + k0 / 2) = q;
-      if ((lane & 3) == 0) scales[mma_scale_offset(row, k0 / 32, K / 128)] = (uint8_t)code;
+      g = gamma[e];
+    } else {
+      g = gamma[0];
     }
+    const int k0 = c * 1024 + lane * 32;
+    if (k0 >= K) continue;
+    float v[32];
+    load32_bf16(x + t * K + k0, v);
+    const uint32_t code = quantize_block32(v, g, codes + row * (K / 2) + k0 / 2);
+    scales[mma_scale_offset(row, k0 / 32, K / 128)] = (uint8_t)code;
   }
 }
 
-// SwiGLU + requantisation: one warp task = (slot, 256 outputs); the slot's
-// expert and row come from the routing arrays.
+// SwiGLU + requantisation: one warp task = (slot, 1024 outputs), lane l the
+// scale block [1024 c + 32 l, +32) of h; the slot's expert and row come from
+// the routing arrays.  With amax_bits set (calibration) the per-expert amax
+// of h is accumulated instead.
 __global__ void __launch_bounds__(256) swiglu_quant_kernel(const uint16_t* __restrict__ y_gu, int I, int R, int E,
                                                            const int32_t* __restrict__ topk_ids,
                                                            const int32_t* __restrict__ slot_to_row, int rows_cap,
@@ -93,7 +88,7 @@ __global__ void __launch_bounds__(256) swiglu_quant_kernel(const uint16_t* __res
                                                            uint8_t* __restrict__ h_codes, uint8_t* __restrict__ h_scales,
                                                            unsigned int* __restrict__ amax_bits) {
   const int lane = threadIdx.x & 31;
-  const int chunks = I / 256;
+  const int chunks = (I + 1023) / 1024;
   const int64_t ntasks = (int64_t)R * chunks;
   const int64_t wstride = (int64_t)gridDim.x * (blockDim.x >> 5);
   for (int64_t task = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); task < ntasks; task += wstride) {
@@ -105,32 +100,42 @@ __global__ void __launch_bounds__(256) swiglu_quant_kernel(const uint16_t* __res
       if (lane == 0) record_error(kWhereSwiglu, kErrFault);
       continue;
     }
-    const int i0 = c * 256 + lane * 8;
-    float g[8], u[8], h[8];
-    load8_bf16(y_gu + row * (2 * I) + i0, g);
-    load8_bf16(y_gu + row * (2 * I) + I + i0, u);
+    const int i0 = c * 1024 + lane * 32;
+    const bool active = i0 < I;
+    float h[32];
+    if (active) {
+      float u[32];
+      load32_bf16(y_gu + row * (2 * I) + i0, h);          // gate
+      load32_bf16(y_gu + row * (2 * I) + I + i0, u);      // up
+      // SiLU(g) = g / (1 + e^-g) in binary32 with the hardware exponential
+      // and divide (a few ulp; for g < -88 the denominator overflows and
+      // the quotient is 0)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float sg = __fdiv_rn(g[i], __fadd_rn(1.0f, expf(-g[i])));
-      h[i] = __fmul_rn(sg, u[i]);
+      for (int i = 0; i < 32; ++i) {
+        const float sg = __fdividef(h[i], __fadd_rn(1.0f, __expf(-h[i])));
+        h[i] = __fmul_rn(sg, u[i]);
+      }
     }
     if (amax_bits) {             // calibration: per-expert amax of h
       float a = 0.0f;
+      if (active) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(h[i]));
+        for (int i = 0; i < 32; ++i) a = fmaxf(a, fabsf(h[i]));
+      }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
       if (lane == 0) atomicMax(amax_bits + e, __float_as_uint(a));
       continue;
     }
-    uint32_t code;
-    const uint32_t q = quantize_lane8(h, gamma_h[e], &code);
-    *reinterpret_cast<uint32_t*>(h_codes + row * (I / 2) + i0 / 2) = q;
-    if ((lane & 3) == 0) h_scales[mma_scale_offset(row, i0 / 32, I / 128)] = (uint8_t)code;
+    if (!active) continue;
+    const uint32_t code = quantize_block32(h, gamma_h[e], h_codes + row * (I / 2) + i0 / 2);
+    h_scales[mma_scale_offset(row, i0 / 32, I / 128)] = (uint8_t)code;
   }
 }
 
-// Router-weighted combine: one warp task = (token, 256 columns).
+// Router-weighted combine: one warp task = (token, 256 columns).  Lane j < k
+// fetches slot j's row and weight; the rows of up to 8 slots are then loaded
+// together and summed in slot order (fp32, j = 0 .. k-1).
 __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ y, int H, int T, int k,
                                                       const float* __restrict__ topk_w,
                                                       const int32_t* __restrict__ slot_to_row, int rows_cap,
@@ -142,17 +147,42 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
   for (int64_t task = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); task < ntasks; task += wstride) {
     const int64_t t = task / chunks;
     const int h0 = (int)(task % chunks) * 256 + lane * 8;
-    if (h0 >= H) continue;
-    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int j = 0; j < k; ++j) {
-      const int64_t row = slot_to_row[t * k + j];
-      if (row < 0 || row >= rows_cap) { record_error(kWhereCombine, kErrFault); continue; }
-      const float w = topk_w[t * k + j];
-      float v[8];
-      load8_bf16(y + row * H + h0, v);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], __fmul_rn(w, v[i]));
+    const bool active = h0 < H;
+    int my_row = -1;
+    float my_w = 0.0f;
+    if (lane < k) {
+      my_row = slot_to_row[t * k + lane];
+      my_w = topk_w[t * k + lane];
     }
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int j0 = 0; j0 < k; j0 += 8) {
+      uint4 raw[8];
+      int rows[8];
+      float ws[8];
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        rows[jj] = __shfl_sync(0xffffffffu, my_row, (j0 + jj) & 31);
+        ws[jj] = __shfl_sync(0xffffffffu, my_w, (j0 + jj) & 31);
+        raw[jj] = make_uint4(0u, 0u, 0u, 0u);
+        if (active && j0 + jj < k && rows[jj] >= 0 && rows[jj] < rows_cap)
+          raw[jj] = __ldg(reinterpret_cast<const uint4*>(y + (int64_t)rows[jj] * H + h0));
+      }
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        if (j0 + jj >= k) break;
+        if (rows[jj] < 0 || rows[jj] >= rows_cap) {
+          if (lane == 0) record_error(kWhereCombine, kErrFault);
+          continue;
+        }
+        const uint32_t wd[4] = {raw[jj].x, raw[jj].y, raw[jj].z, raw[jj].w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float v = (i & 1) ? bf16hi(wd[i >> 1]) : bf16lo(wd[i >> 1]);
+          acc[i] = __fadd_rn(acc[i], __fmul_rn(ws[jj], v));
+        }
+      }
+    }
+    if (!active) continue;
     uint4 o;
     o.x = f32_to_bf16_bits(acc[0]) | (f32_to_bf16_bits(acc[1]) << 16);
     o.y = f32_to_bf16_bits(acc[2]) | (f32_to_bf16_bits(acc[3]) << 16);

@@ -205,7 +205,9 @@ moesq_status moesq_route_permute_noalloc(const float* logits, const moesq_routin
  * with gamma[rt->topk_ids[t*k+j]], to row rt->slot_to_row[t*k+j] (the fused
  * dispatch-scatter + quantisation of App. D.1); rows_cap = rt->rows_cap.
  * Plain form (rt == NULL): token t goes to row t with gamma[0]; rows_cap is
- * the allocated row count (multiple of 128, >= T).                       */
+ * the allocated row count (multiple of 128, >= T).
+ * K is a multiple of 256; x_bf16 and codes are 16-byte aligned
+ * (MOESQ_ERR_INVALID_ARG otherwise).                                      */
 moesq_status moesq_quantize_act(const uint16_t* x_bf16, int T, int K,
                                 const moesq_routing* rt, const float* gamma,
                                 int rows_cap, uint8_t* codes, uint8_t* scales,
@@ -243,9 +245,11 @@ moesq_status moesq_grouped_sparse_gemm(const moesq_weights* w, const uint8_t* a_
 /* ------------------------------------------------------------- layer parts
  * moesq_swiglu_quant: h = SiLU(g) * u for every valid row of the gate_up
  * output y_gu [rows_cap][2I] bf16 (g = columns [0, I), u = [I, 2I);
- * SiLU(g) = g / (1 + e^-g), binary32), requantised to NVFP4 with
+ * SiLU(g) = g / (1 + e^-g) in binary32 with the hardware exponential and
+ * divide, a few ulp from the exact value), requantised to NVFP4 with
  * gamma_h[e] of the row's expert into h_codes [rows_cap][I/2] and h_scales
- * (MMA scale layout) -- the fused SwiGLU + requantisation of App. D.1. */
+ * (MMA scale layout) -- the fused SwiGLU + requantisation of App. D.1.
+ * I is a multiple of 256; y_gu and h_codes are 16-byte aligned. */
 moesq_status moesq_swiglu_quant(const uint16_t* y_gu, int I, const moesq_routing* rt,
                                 const float* gamma_h, uint8_t* h_codes, uint8_t* h_scales,
                                 void* stream);

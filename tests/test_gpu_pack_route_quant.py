@@ -145,3 +145,106 @@ def test_swiglu_quant_matches_oracle(cuda_lib):
     # an exact rounding boundary; scales and almost all codes agree
     assert (gs == os_).mean() > 0.999
     assert (gc == oc).mean() > 0.999
+
+
+# ---------------------------------------------------------------- quantiser near the E2M1 decision points
+E2M1_DECISIONS = (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0)   # midpoints of the E2M1 grid (App. A, Fig. 3)
+
+
+def _bf16_neighbours(t: np.ndarray):
+    """The bf16 numbers just below-or-at and just above t > 0 (exact in float64)."""
+    e = np.floor(np.log2(t))
+    ulp = 2.0 ** (e - 7)
+    lo = np.floor(t / ulp) * ulp
+    return lo, lo + ulp
+
+
+def _boundary_rows(gamma: float, T: int, K: int, rng):
+    """Rows whose blocks hold an amax A and, for every decision point tau, the
+    bf16 values nearest tau * s_b (both signs), s_b = UE4M3(code_b) / gamma."""
+    nb = K // 32
+    amax = rng.uniform(1.0, 2.0, size=(T, nb)) * 2.0 ** rng.integers(-3, 6, size=(T, nb))
+    a_bits = S.f32_to_bf16_bits_np(amax.astype(np.float32))
+    only_a = np.zeros((T, K), np.uint16)
+    only_a[:, ::32] = a_bits
+    _, sc = O.quantize_rows_bf16(only_a, gamma)
+    s = (np.array([O.ue4m3_value(int(c)) for c in sc.ravel()], np.float32).reshape(T, nb)
+         / np.float32(gamma)).astype(np.float64)
+    vals = np.zeros((T, nb, 32), np.float64)
+    taus = np.zeros((T, nb, 32), np.float64)
+    j = 1
+    for tau in E2M1_DECISIONS:
+        lo, hi = _bf16_neighbours(tau * s)
+        for v in (lo, hi):
+            vals[:, :, j], taus[:, :, j] = v, tau
+            vals[:, :, j + 1], taus[:, :, j + 1] = -v, tau
+            j += 2
+    x = S.f32_to_bf16_bits_np(vals.astype(np.float32)).reshape(T, nb, 32)
+    x[:, :, 0] = a_bits
+    rel = np.abs(np.abs(vals[:, :, 1:j]) / (s[:, :, None] * taus[:, :, 1:j]) - 1.0)
+    return x.reshape(T, K), rel
+
+
+@pytest.mark.parametrize("gamma", [1.0, 0.125, 32.0, 3.7, 259.1])
+def test_quantize_near_decision_points_bit_exact(cuda_lib, gamma):
+    """Every value within one bf16 step of an E2M1 decision point (exact ties
+    when the step is a power of two): the GPU codes equal the oracle's, which
+    rounds the correctly rounded quotient."""
+    m = cuda_lib
+    T, K = 64, 512
+    rng = np.random.default_rng(int(gamma * 1000) + 7)
+    x, rel = _boundary_rows(np.float32(gamma), T, K, rng)
+    g = np.float32(gamma)
+    oc, os_ = O.quantize_rows_bf16(x, g)
+    rc = 128
+    codes, scales = m.act_buffers(rc, K)
+    m.moesq_quantize_act(to_dev(x), T, K, None, to_dev(np.array([g], np.float32)), rc, codes, scales)
+    assert (L.mma_to_scales(to_np(scales), rc, K)[:T] == os_).all()
+    assert (to_np(codes)[:T] == oc).all()
+    if gamma in (1.0, 0.125, 32.0):
+        assert (rel == 0).sum() > 100                      # exact ties on the decision points
+
+
+def _near_miss_case(rng):
+    """A global scale gamma, block amax A and bf16 value v with v / s_b within
+    2^-21 (relative, nonzero) of a decision point, s_b = UE4M3(code) / gamma."""
+    while True:
+        c = int(rng.integers(40, 110))
+        tau = float(rng.choice(E2M1_DECISIONS))
+        v = float(np.frombuffer((np.uint32(S.f32_to_bf16_bits_np(np.float32([rng.uniform(1, 2)]))[0]) << 16).tobytes(),
+                                np.float32)[0])
+        val = O.ue4m3_value(c)
+        g0 = np.float32(tau * val / v)
+        want_above = bool(rng.integers(0, 2))
+        for step in range(-64, 65):
+            g = np.float32(g0 * (1.0 + step * 2.0 ** -23))
+            sb = np.float32(np.float32(val) / g)
+            d = (v / float(sb)) / tau - 1.0
+            if d != 0 and abs(d) < 2.0 ** -21 and (d > 0) == want_above:
+                amax = float(np.float32(6.0 * val / float(g)))
+                a_bits = S.f32_to_bf16_bits_np(np.float32([amax]))[0]
+                _, sc = O.quantize_rows_bf16(np.array([[a_bits] + [0] * 31], np.uint16), g)
+                if int(sc[0, 0]) == c:
+                    return g, a_bits, v
+                break
+
+
+def test_quantize_guard_band_bit_exact(cuda_lib):
+    """Quotients within 2^-21 of a decision point (above and below), where the
+    fast reciprocal path must defer to the exact quotient."""
+    m = cuda_lib
+    rng = np.random.default_rng(2024)
+    T, K = 8, 256
+    for _ in range(24):
+        g, a_bits, v = _near_miss_case(rng)
+        vb = S.f32_to_bf16_bits_np(np.float32([v, -v]))
+        x = np.zeros((T, K), np.uint16)
+        x[:, ::32] = a_bits
+        for j in range(1, 32, 2):
+            x[:, j::32] = vb[0]
+            x[:, j + 1::32] = vb[1] if j + 1 < 32 else 0
+        oc, os_ = O.quantize_rows_bf16(x, g)
+        codes, scales = m.act_buffers(128, K)
+        m.moesq_quantize_act(to_dev(x), T, K, None, to_dev(np.array([g], np.float32)), 128, codes, scales)
+        assert (L.mma_to_scales(to_np(scales), 128, K)[:T] == os_).all()
+        assert (to_np(codes)[:T] == oc).all()
