@@ -59,6 +59,15 @@ WORKLOADS = {
     "kimi_down_t8192_zipf": (384, 8, 7168, 2048, 8192, "zipf", "gemm_down"),
     "30b_gateup_t256": (128, 8, 2048, 768, 256, "uniform", "gemm"),
 }
+# The paper's Table 11 setting (App. D, B200): Kimi gate_up over all 384
+# experts, expert g receiving N * {1, 3/4, 1/2, 1/4}[g % 4] rows, timed as
+# activation quantisation + grouped GEMM (bf16 in, bf16 out); the step is
+# those two calls.  Value: the paper's latency in us and its effective
+# TFLOP/s (2 M K sum(n) / t).
+TAB11 = {8: (760.0, 148.0), 16: (793.0, 284.0), 32: (843.0, 535.0), 64: (925.0, 975.0),
+         128: (912.0, 1978.0), 256: (1370.0, 2633.0)}
+for _n in TAB11:
+    WORKLOADS["tab11_n%d" % _n] = (384, 8, 7168, 2048, 30 * _n, "tab11", "quant_gemm")
 DEFAULT_WORKLOAD = "30b_layer_t256"
 
 
@@ -160,7 +169,7 @@ def step_work(E, k, H, I, T, counts_gu, kind):
     gu_w = touched * packed_weight_bytes(2 * I, H)
     gu_bytes = gu_w + R * (H // 2 + H // 32) + R * 2 * I * 2
     gu_fl = 2.0 * 2 * I * H * R
-    if kind == "gemm":
+    if kind in ("gemm", "quant_gemm"):
         return gu_fl, gu_w, {"gate_up": gu_bytes}, {"gate_up": gu_fl}
     dn_w = touched * packed_weight_bytes(H, I)
     dn_bytes = dn_w + R * (I // 2 + I // 32) + R * H * 2
@@ -191,7 +200,25 @@ def job_throughput(flops_per_rank, world, ms):
     return world * flops_per_rank / (ms * 1e-3) / 1e12
 
 
+def tab11_logits(T, E, k=8):
+    """0/1 router logits whose top-k gives expert g exactly
+    N * {4, 3, 2, 1}[g % 4] / 4 rows (N = T / 30): every token takes the k
+    experts with the most rows still to fill (ties to the lower id)."""
+    n = T // 30
+    left = np.array([n * (4 - g % 4) // 4 for g in range(E)], np.int64)
+    assert left.sum() == T * k
+    lg = np.zeros((T, E), np.float32)
+    for t in range(T):
+        pick = np.lexsort((np.arange(E), -left))[:k]
+        assert (left[pick] > 0).all()
+        lg[t, pick] = 1.0
+        left[pick] -= 1
+    return lg
+
+
 def logits_for(routing, seed, T, E):
+    if routing == "tab11":
+        return tab11_logits(T, E)
     return S.zipf_logits_np(seed, T, E) if routing == "zipf" else S.uniform_logits_np(seed, T, E)
 
 
@@ -260,7 +287,12 @@ def run_cuda(args, rank, world, local_rank):
     def c_gemm_main():
         m.moesq_grouped_sparse_gemm(w_main, a_codes, a_scales, rb.rows_cap, rb.counts, rb.row_offsets, ga, y_main)
 
-    comps = [("route_quant", c_route_quant), ("gemm_main", c_gemm_main)]
+    if kind == "quant_gemm":                  # fixed grouping: routed once, outside the step
+        m.moesq_route_permute(lg, rb)
+        comps = [("quant", lambda: m.moesq_quantize_act(x, T, K_in, rb, ga, rb.rows_cap, a_codes, a_scales)),
+                 ("gemm_main", c_gemm_main)]
+    else:
+        comps = [("route_quant", c_route_quant), ("gemm_main", c_gemm_main)]
     if kind == "layer":
         comps += [("swiglu_quant", lambda: m.moesq_swiglu_quant(y_main, I, rb, gh, h_codes, h_scales)),
                   ("gemm_down", lambda: m.moesq_grouped_sparse_gemm(w_dn, h_codes, h_scales, rb.rows_cap, rb.counts,
@@ -272,7 +304,7 @@ def run_cuda(args, rank, world, local_rank):
             f()
 
     # routing: one fused kernel for T <= 128 tokens, else top-k, count, scan and scatter
-    launches_per_step = (1 if T <= 128 else 4) + 2 + (3 if kind == "layer" else 0)
+    launches_per_step = (0 if kind == "quant_gemm" else 1 if T <= 128 else 4) + 2 + (3 if kind == "layer" else 0)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
         flush.zero_()
@@ -413,7 +445,7 @@ def run_oracle_sample(workload, n_tokens, seed=1234):
         O.grouped_gemm(pk, a_c, a_s, rt.offsets, ga)
         return time.perf_counter() - t0, 2.0 * H * I * n * k
     pk_gu = packed(0, 2 * I, H)
-    if kind == "gemm":
+    if kind in ("gemm", "quant_gemm"):
         t0 = time.perf_counter()
         rt = O.route(lg, k)
         a_c, a_s = O.permute_quantize(x, rt, ga)
@@ -429,7 +461,7 @@ def run_oracle_sample(workload, n_tokens, seed=1234):
 def oracle_sample_tokens(workload):
     """Token sample sized for roughly 10-30 s of single-threaded oracle time."""
     E, k, H, I, T, routing, kind = WORKLOADS[workload]
-    per_token_macs = k * (3 * I * H if kind == "layer" else 2 * I * H if kind == "gemm" else H * I)
+    per_token_macs = k * (3 * I * H if kind == "layer" else 2 * I * H if kind in ("gemm", "quant_gemm") else H * I)
     return max(1, min(T, int(2.5e9 // per_token_macs)))
 
 
@@ -516,9 +548,11 @@ def main():
                      "hbm_frac": hbm_ach / hbm_peak, "tensor_frac": tc_ach / tc_peak,
                      "peak_source": "%s (tensor peak = dense bf16 burst x %g fp4/bf16 x %g sparse)"
                      % (peaks["source"], FP4_OVER_BF16, SPARSE_FACTOR)})
+    tab11_n = T // 30 if args.workload.startswith("tab11_") else None
+    vs_baseline = value / TAB11[tab11_n][1] if tab11_n else None
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "nvfp4 (e2m1 x ue4m3 products, f32 accumulate, bf16 out)",
+            "vs_baseline": vs_baseline, "dtype": "nvfp4 (e2m1 x ue4m3 products, f32 accumulate, bf16 out)",
             "data": "synthetic (seeded; pages' shapes and distributions)", "config": config,
             "weight_gbs": weight_gbs, "breakdown_ms": r["parts"], "roofline": roofline,
             "clocks": r["clocks"], "gpu_launches": r["launches"],
