@@ -303,8 +303,8 @@ def run_cuda(args, rank, world, local_rank):
         for _, f in comps:
             f()
 
-    # routing: one fused kernel for T <= 128 tokens, else top-k, count, scan and scatter
-    launches_per_step = (0 if kind == "quant_gemm" else 1 if T <= 128 else 4) + 2 + (3 if kind == "layer" else 0)
+    # routing: top-k plus one finishing kernel for T <= 512 tokens, else top-k, count, scan and scatter
+    launches_per_step = (0 if kind == "quant_gemm" else 2 if T <= 512 else 4) + 2 + (3 if kind == "layer" else 0)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
         flush.zero_()

@@ -228,15 +228,15 @@ template <int PL>
 moesq_status route_launch_pl(const float* logits, const moesq_routing* rt, int32_t* bc, cudaStream_t s) {
   const int nblk = (rt->T + kRouteTPB - 1) / kRouteTPB;
   const size_t smem = (size_t)rt->E * kRouteWords * 4;
-  if (rt->T <= kRouteSmallMaxT) {       // few tokens: fused single-CTA path
+  route_topk_kernel<PL><<<(rt->T + 7) / 8, 256, 0, s>>>(logits, rt->T, rt->E, rt->k, rt->topk_ids, rt->topk_w);
+  MOESQ_TRY(last_launch());
+  if (rt->T <= kRouteSmallMaxT) {       // few tokens: one CTA counts, scans and scatters
     const int words = (rt->T + 31) / 32;
-    route_small_kernel<PL><<<1, 1024, (size_t)rt->E * words * 4, s>>>(
+    route_small_kernel<PL, false><<<1, 1024, (size_t)rt->E * words * 4, s>>>(
         logits, rt->T, rt->E, rt->k, rt->topk_ids, rt->topk_w, rt->counts, rt->offsets, rt->row_offsets,
         rt->sorted_to_slot, rt->slot_to_row, words);
     return last_launch();
   }
-  route_topk_kernel<PL><<<(rt->T + 7) / 8, 256, 0, s>>>(logits, rt->T, rt->E, rt->k, rt->topk_ids, rt->topk_w);
-  MOESQ_TRY(last_launch());
   route_count_kernel<<<nblk, 256, smem, s>>>(rt->T, rt->E, rt->k, rt->topk_ids, bc);
   MOESQ_TRY(last_launch());
   route_scan_kernel<<<1, 1024, 0, s>>>(bc, nblk, rt->E, rt->counts, rt->offsets, rt->row_offsets);

@@ -10,7 +10,7 @@ namespace moesq {
 
 constexpr int kRouteTPB = 128;          // tokens per routing block
 constexpr int kRouteWords = kRouteTPB / 32;
-constexpr int kRouteSmallMaxT = 128;     // tokens routed by the single-CTA kernel
+constexpr int kRouteSmallMaxT = 512;     // tokens whose counts / scan / scatter one CTA does
 constexpr int kRouteMaxE = 512;
 constexpr int kRouteMaxPerLane = kRouteMaxE / 32;
 
@@ -199,10 +199,11 @@ __global__ void __launch_bounds__(256) route_scatter_kernel(int T, int E, int k,
   }
 }
 
-// Single-CTA routing for T <= kRouteSmallMaxT tokens: top-k, counts, offsets
-// and the scatter in one launch, with the same arithmetic as the multi-kernel
-// path; the expert bitmaps hold words = ceil(T / 32) words each.
-template <int PL>
+// Single-CTA routing for few tokens: counts, offsets and the scatter (and,
+// with kTopk, the top-k itself) in one launch, with the same arithmetic as
+// the multi-kernel path; the expert bitmaps hold words = ceil(T / 32) words
+// each.  Without kTopk the ids come from route_topk_kernel.
+template <int PL, bool kTopk>
 __global__ void __launch_bounds__(1024) route_small_kernel(const float* __restrict__ logits, int T, int E, int k,
                                                            int32_t* __restrict__ topk_ids, float* __restrict__ topk_w,
                                                            int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
@@ -216,9 +217,16 @@ __global__ void __launch_bounds__(1024) route_small_kernel(const float* __restri
   for (int i = threadIdx.x; i < E * words; i += blockDim.x) bitmap[i] = 0;
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-  for (int tl = warp; tl < T; tl += nwarps)
-    topk_one_token<PL>(logits + (size_t)tl * E, E, k, lane, topk_ids + (size_t)tl * k, topk_w + (size_t)tl * k,
-                       bitmap, words, tl);
+  if (kTopk) {
+    for (int tl = warp; tl < T; tl += nwarps)
+      topk_one_token<PL>(logits + (size_t)tl * E, E, k, lane, topk_ids + (size_t)tl * k, topk_w + (size_t)tl * k,
+                         bitmap, words, tl);
+  } else {                               // ids from route_topk_kernel: set the bitmaps
+    for (int i = threadIdx.x; i < T * k; i += blockDim.x) {
+      const int e = topk_ids[i], tl = i / k;
+      if (e >= 0 && e < E) atomicOr(&bitmap[e * words + (tl >> 5)], 1u << (tl & 31));
+    }
+  }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int c = 0;
