@@ -150,6 +150,9 @@ grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const GemmP
     tmem_alloc(smem_u32(misc), C::kTmemCols);
     tmem_relinquish();
   }
+  // the routing counts come from the previous kernels of the step
+  pdl_trigger();
+  pdl_wait();
   // expert table; validate the routing counts against the aligned row space
   int local_bad = 0;
   for (int e = threadIdx.x; e < E; e += blockDim.x) {

@@ -9,6 +9,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "../../include/moesq.h"
 #include "common.cuh"
@@ -48,6 +49,28 @@ thread_local cudaError_t t_last_cuda_error = cudaSuccess;
 
 inline moesq_status last_launch() {
   const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) return MOESQ_OK;
+  t_last_cuda_error = e;
+  return MOESQ_ERR_CUDA;
+}
+
+// Launch with programmatic stream serialisation: the grid may start while its
+// predecessor in the stream finishes; every such kernel calls
+// griddepcontrol.wait before it touches global memory.
+template <typename... KArgs, typename... Args>
+moesq_status launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                        Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
   if (e == cudaSuccess) return MOESQ_OK;
   t_last_cuda_error = e;
   return MOESQ_ERR_CUDA;
@@ -153,8 +176,7 @@ moesq_status launch_gemm(const moesq_weights* w, const uint8_t* a_codes, const u
   p.rows_cap = rows_cap;
   p.timeout_ns = g_timeout_ns;
   const int grid = num_ctas > 0 ? num_ctas : di.sms * C::kCtasPerSm;
-  grouped_sparse_gemm_kernel<TN><<<grid, kGemmThreads, C::kSmemBytes, s>>>(tmb, p);
-  return last_launch();
+  return launch_pdl(grouped_sparse_gemm_kernel<TN>, dim3(grid), dim3(kGemmThreads), (size_t)C::kSmemBytes, s, tmb, p);
 }
 
 // Layer workspace carve-up.
@@ -228,22 +250,19 @@ template <int PL>
 moesq_status route_launch_pl(const float* logits, const moesq_routing* rt, int32_t* bc, cudaStream_t s) {
   const int nblk = (rt->T + kRouteTPB - 1) / kRouteTPB;
   const size_t smem = (size_t)rt->E * kRouteWords * 4;
-  route_topk_kernel<PL><<<(rt->T + 7) / 8, 256, 0, s>>>(logits, rt->T, rt->E, rt->k, rt->topk_ids, rt->topk_w);
-  MOESQ_TRY(last_launch());
+  MOESQ_TRY(launch_pdl(route_topk_kernel<PL>, dim3((rt->T + 7) / 8), dim3(256), 0, s, logits, rt->T, rt->E, rt->k,
+                       rt->topk_ids, rt->topk_w));
   if (rt->T <= kRouteSmallMaxT) {       // few tokens: one CTA counts, scans and scatters
     const int words = (rt->T + 31) / 32;
-    route_small_kernel<PL, false><<<1, 1024, (size_t)rt->E * words * 4, s>>>(
-        logits, rt->T, rt->E, rt->k, rt->topk_ids, rt->topk_w, rt->counts, rt->offsets, rt->row_offsets,
-        rt->sorted_to_slot, rt->slot_to_row, words);
-    return last_launch();
+    return launch_pdl(route_small_kernel<PL, false>, dim3(1), dim3(1024), (size_t)rt->E * words * 4, s, logits,
+                      rt->T, rt->E, rt->k, rt->topk_ids, rt->topk_w, rt->counts, rt->offsets, rt->row_offsets,
+                      rt->sorted_to_slot, rt->slot_to_row, words);
   }
-  route_count_kernel<<<nblk, 256, smem, s>>>(rt->T, rt->E, rt->k, rt->topk_ids, bc);
-  MOESQ_TRY(last_launch());
-  route_scan_kernel<<<1, 1024, 0, s>>>(bc, nblk, rt->E, rt->counts, rt->offsets, rt->row_offsets);
-  MOESQ_TRY(last_launch());
-  route_scatter_kernel<<<nblk, 256, smem, s>>>(rt->T, rt->E, rt->k, rt->topk_ids, bc, rt->offsets, rt->row_offsets,
-                                               rt->sorted_to_slot, rt->slot_to_row);
-  return last_launch();
+  MOESQ_TRY(launch_pdl(route_count_kernel, dim3(nblk), dim3(256), smem, s, rt->T, rt->E, rt->k, rt->topk_ids, bc));
+  MOESQ_TRY(launch_pdl(route_scan_kernel, dim3(1), dim3(1024), 0, s, bc, nblk, rt->E, rt->counts, rt->offsets,
+                       rt->row_offsets));
+  return launch_pdl(route_scatter_kernel, dim3(nblk), dim3(256), smem, s, rt->T, rt->E, rt->k, rt->topk_ids, bc,
+                    rt->offsets, rt->row_offsets, rt->sorted_to_slot, rt->slot_to_row);
 }
 
 moesq_status route_launch(const float* logits, const moesq_routing* rt, int32_t* bc, cudaStream_t s) {
@@ -430,9 +449,8 @@ moesq_status moesq_quantize_act(const uint16_t* x_bf16, int T, int K, const moes
   }
   cudaStream_t s = as_stream(stream);
   const int64_t tasks = (int64_t)T * k * ((K + 1023) / 1024);
-  quantize_act_kernel<<<grid_for(tasks, 8, device_info().sms), 256, 0, s>>>(x_bf16, T, K, k, ids, s2r, E, gamma,
-                                                                            rows_cap, codes, scales);
-  return last_launch();
+  return launch_pdl(quantize_act_kernel, dim3(grid_for(tasks, 8, device_info().sms)), dim3(256), 0, s, x_bf16, T, K,
+                    k, ids, s2r, E, gamma, rows_cap, codes, scales);
 }
 
 moesq_status moesq_act_global_scale(const uint16_t* x_bf16, int64_t n, float* gamma_out, void* stream) {
@@ -478,9 +496,9 @@ moesq_status moesq_swiglu_quant(const uint16_t* y_gu, int I, const moesq_routing
   if (!aligned(y_gu, 16) || !aligned(h_codes, 16)) return MOESQ_ERR_INVALID_ARG;
   const int R = rt->T * rt->k;
   const int64_t tasks = (int64_t)R * ((I + 1023) / 1024);
-  swiglu_quant_kernel<<<grid_for(tasks, 8, device_info().sms), 256, 0, as_stream(stream)>>>(
-      y_gu, I, R, rt->E, rt->topk_ids, rt->slot_to_row, rt->rows_cap, gamma_h, h_codes, h_scales, nullptr);
-  return last_launch();
+  return launch_pdl(swiglu_quant_kernel, dim3(grid_for(tasks, 8, device_info().sms)), dim3(256), 0, as_stream(stream),
+                    y_gu, I, R, rt->E, rt->topk_ids, rt->slot_to_row, rt->rows_cap, gamma_h, h_codes, h_scales,
+                    (unsigned int*)nullptr);
 }
 
 moesq_status moesq_combine(const uint16_t* y, int H, const moesq_routing* rt, uint16_t* out, void* stream) {
@@ -488,9 +506,8 @@ moesq_status moesq_combine(const uint16_t* y, int H, const moesq_routing* rt, ui
   if (!y || !out || H < 8 || H % 8) return MOESQ_ERR_INVALID_ARG;
   if (!aligned(y, 16) || !aligned(out, 16)) return MOESQ_ERR_INVALID_ARG;
   const int64_t tasks = (int64_t)rt->T * ((H + 255) / 256);
-  combine_kernel<<<grid_for(tasks, 8, device_info().sms), 256, 0, as_stream(stream)>>>(
-      y, H, rt->T, rt->k, rt->topk_w, rt->slot_to_row, rt->rows_cap, out);
-  return last_launch();
+  return launch_pdl(combine_kernel, dim3(grid_for(tasks, 8, device_info().sms)), dim3(256), 0, as_stream(stream), y,
+                    H, rt->T, rt->k, rt->topk_w, rt->slot_to_row, rt->rows_cap, out);
 }
 
 size_t moesq_layer_workspace_bytes(int T, int k, int E, int H, int I) {

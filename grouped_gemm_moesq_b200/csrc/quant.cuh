@@ -46,6 +46,8 @@ __global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t* __res
                                                            const int32_t* __restrict__ slot_to_row, int E,
                                                            const float* __restrict__ gamma, int rows_cap,
                                                            uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int chunks = (K + 1023) / 1024;
   const int nslots = slot_to_row ? k : 1;
@@ -87,6 +89,8 @@ __global__ void __launch_bounds__(256) swiglu_quant_kernel(const uint16_t* __res
                                                            const float* __restrict__ gamma_h,
                                                            uint8_t* __restrict__ h_codes, uint8_t* __restrict__ h_scales,
                                                            unsigned int* __restrict__ amax_bits) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int chunks = (I + 1023) / 1024;
   const int64_t ntasks = (int64_t)R * chunks;
@@ -140,6 +144,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
                                                       const float* __restrict__ topk_w,
                                                       const int32_t* __restrict__ slot_to_row, int rows_cap,
                                                       uint16_t* __restrict__ out) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int chunks = (H + 255) / 256;
   const int64_t ntasks = (int64_t)T * chunks;

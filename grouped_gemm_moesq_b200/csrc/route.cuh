@@ -80,6 +80,8 @@ __device__ __forceinline__ void topk_one_token(const float* __restrict__ lr, int
 template <int PL>
 __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
                                                          int32_t* __restrict__ topk_ids, float* __restrict__ topk_w) {
+  pdl_trigger();
+  pdl_wait();
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
   topk_one_token<PL>(logits + (size_t)t * E, E, k, threadIdx.x & 31, topk_ids + (size_t)t * k,
@@ -89,6 +91,8 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
 // K1b: per 128-token block, per-expert counts from the block's token bitmaps.
 __global__ void __launch_bounds__(256) route_count_kernel(int T, int E, int k, const int32_t* __restrict__ topk_ids,
                                                           int32_t* __restrict__ block_counts) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ uint32_t bitmap[];                 // [E][kRouteWords]
   for (int i = threadIdx.x; i < E * kRouteWords; i += blockDim.x) bitmap[i] = 0;
   __syncthreads();
@@ -113,6 +117,8 @@ __global__ void __launch_bounds__(256) route_count_kernel(int T, int E, int k, c
 __global__ void __launch_bounds__(1024) route_scan_kernel(int32_t* __restrict__ block_counts, int nblk, int E,
                                                           int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                                                           int32_t* __restrict__ row_offsets) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int32_t s_cnt[kRouteMaxE];
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int run = 0;
@@ -171,6 +177,8 @@ __global__ void __launch_bounds__(256) route_scatter_kernel(int T, int E, int k,
                                                             const int32_t* __restrict__ row_offsets,
                                                             int32_t* __restrict__ sorted_to_slot,
                                                             int32_t* __restrict__ slot_to_row) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ uint32_t bitmap[];                 // [E][kRouteWords]
   for (int i = threadIdx.x; i < E * kRouteWords; i += blockDim.x) bitmap[i] = 0;
   __syncthreads();
@@ -210,6 +218,8 @@ __global__ void __launch_bounds__(1024) route_small_kernel(const float* __restri
                                                            int32_t* __restrict__ row_offsets,
                                                            int32_t* __restrict__ sorted_to_slot,
                                                            int32_t* __restrict__ slot_to_row, int words) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ uint32_t bitmap[];                 // [E][words]
   __shared__ int32_t s_cnt[kRouteMaxE];
   __shared__ int32_t s_off[kRouteMaxE];
