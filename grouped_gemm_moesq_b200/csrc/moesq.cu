@@ -254,9 +254,9 @@ moesq_status route_launch_pl(const float* logits, const moesq_routing* rt, int32
                        rt->topk_ids, rt->topk_w));
   if (rt->T <= kRouteSmallMaxT) {       // few tokens: one CTA counts, scans and scatters
     const int words = (rt->T + 31) / 32;
-    return launch_pdl(route_small_kernel<PL, false>, dim3(1), dim3(1024), (size_t)rt->E * words * 4, s, logits,
-                      rt->T, rt->E, rt->k, rt->topk_ids, rt->topk_w, rt->counts, rt->offsets, rt->row_offsets,
-                      rt->sorted_to_slot, rt->slot_to_row, words);
+    return launch_pdl(route_finish_kernel, dim3(1), dim3(1024), (size_t)rt->E * words * 4, s, rt->T, rt->E, rt->k,
+                      (const int32_t*)rt->topk_ids, rt->counts, rt->offsets, rt->row_offsets, rt->sorted_to_slot,
+                      rt->slot_to_row, words);
   }
   MOESQ_TRY(launch_pdl(route_count_kernel, dim3(nblk), dim3(256), smem, s, rt->T, rt->E, rt->k, rt->topk_ids, bc));
   MOESQ_TRY(launch_pdl(route_scan_kernel, dim3(1), dim3(1024), 0, s, bc, nblk, rt->E, rt->counts, rt->offsets,

@@ -207,17 +207,15 @@ __global__ void __launch_bounds__(256) route_scatter_kernel(int T, int E, int k,
   }
 }
 
-// Single-CTA routing for few tokens: counts, offsets and the scatter (and,
-// with kTopk, the top-k itself) in one launch, with the same arithmetic as
-// the multi-kernel path; the expert bitmaps hold words = ceil(T / 32) words
-// each.  Without kTopk the ids come from route_topk_kernel.
-template <int PL, bool kTopk>
-__global__ void __launch_bounds__(1024) route_small_kernel(const float* __restrict__ logits, int T, int E, int k,
-                                                           int32_t* __restrict__ topk_ids, float* __restrict__ topk_w,
-                                                           int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-                                                           int32_t* __restrict__ row_offsets,
-                                                           int32_t* __restrict__ sorted_to_slot,
-                                                           int32_t* __restrict__ slot_to_row, int words) {
+// Single-CTA finish of the routing for few tokens: from the top-k ids of
+// route_topk_kernel, the expert bitmaps (words = ceil(T / 32) words per
+// expert), counts, offsets and the stable scatter in one launch, with the
+// same arithmetic as the multi-kernel path.
+__global__ void __launch_bounds__(1024) route_finish_kernel(int T, int E, int k, const int32_t* __restrict__ topk_ids,
+                                                            int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                                                            int32_t* __restrict__ row_offsets,
+                                                            int32_t* __restrict__ sorted_to_slot,
+                                                            int32_t* __restrict__ slot_to_row, int words) {
   pdl_trigger();
   pdl_wait();
   extern __shared__ uint32_t bitmap[];                 // [E][words]
@@ -226,16 +224,10 @@ __global__ void __launch_bounds__(1024) route_small_kernel(const float* __restri
   __shared__ int32_t s_roff[kRouteMaxE];
   for (int i = threadIdx.x; i < E * words; i += blockDim.x) bitmap[i] = 0;
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-  if (kTopk) {
-    for (int tl = warp; tl < T; tl += nwarps)
-      topk_one_token<PL>(logits + (size_t)tl * E, E, k, lane, topk_ids + (size_t)tl * k, topk_w + (size_t)tl * k,
-                         bitmap, words, tl);
-  } else {                               // ids from route_topk_kernel: set the bitmaps
-    for (int i = threadIdx.x; i < T * k; i += blockDim.x) {
-      const int e = topk_ids[i], tl = i / k;
-      if (e >= 0 && e < E) atomicOr(&bitmap[e * words + (tl >> 5)], 1u << (tl & 31));
-    }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < T * k; i += blockDim.x) {
+    const int e = topk_ids[i], tl = i / k;
+    if (e >= 0 && e < E) atomicOr(&bitmap[e * words + (tl >> 5)], 1u << (tl & 31));
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {

@@ -233,7 +233,8 @@ moesq_status moesq_act_global_scale(const uint16_t* x_bf16, int64_t n, float* ga
  * cfg may be NULL (defaults).                                            */
 typedef struct {
   int32_t tile_n;      /* token rows per tile: 0 = auto, 64 or 128 */
-  int32_t num_ctas;    /* persistent CTAs: 0 = one per SM */
+  int32_t num_ctas;    /* persistent CTAs: 0 = two per SM (two independent
+                          tensor-core issue streams per SM) */
 } moesq_gemm_config;
 
 moesq_status moesq_grouped_sparse_gemm(const moesq_weights* w, const uint8_t* a_codes,

@@ -62,3 +62,15 @@ def test_job_throughput_counts_all_ranks_over_slowest():
     # 4 ranks, 1e12 dense-equivalent flops each, slowest rank 2 ms
     assert bench.job_throughput(1e12, 4, 2.0) == pytest.approx(2000.0)
     assert bench.rank_seed(7, 0) == 7 and bench.rank_seed(7, 3) != bench.rank_seed(7, 2)
+
+
+def test_tab11_pattern_routes_to_the_paper_counts():
+    """The Table 11 workloads' router logits: top-8 through the oracle's
+    router gives expert g exactly N * {1, 3/4, 1/2, 1/4}[g % 4] rows."""
+    import bench
+    import oracle as O
+    for n in (8, 16):
+        T = 30 * n
+        rt = O.route(bench.tab11_logits(T, 384), 8)
+        want = np.array([n * (4 - g % 4) // 4 for g in range(384)])
+        assert (rt.counts == want).all()
