@@ -67,6 +67,8 @@ def load():
         "moesq_set_wait_timeout_ns": (None, [_c.c_uint64]),
         "moesq_weights_bytes": (_sz, [_c.c_int, _c.c_int, _c.c_int, _P(_sz)]),
         "moesq_pack_weights": (_c.c_int, [_vp, _c.c_int, _c.c_int, _P(moesq_weights), _vp]),
+        "moesq_import_dense_nvfp4": (_c.c_int, [_vp, _vp, _vp, _c.c_int, _c.c_int, _P(moesq_weights), _vp]),
+        "moesq_export_dense_nvfp4": (_c.c_int, [_P(moesq_weights), _vp, _vp]),
         "moesq_rows_capacity": (_i64, [_c.c_int, _c.c_int, _c.c_int]),
         "moesq_route_workspace_bytes": (_sz, [_c.c_int, _c.c_int]),
         "moesq_route_permute": (_c.c_int, [_vp, _P(moesq_routing), _vp, _sz, _vp]),
@@ -206,6 +208,17 @@ def moesq_layer_host_workspace_bytes(T: int, k: int, E: int, H: int, I: int) -> 
 def moesq_pack_weights(w_bf16, e_begin: int, e_count: int, out: PackedWeights, stream=None):
     _check(load().moesq_pack_weights(_ptr(w_bf16), e_begin, e_count, ctypes.byref(out.struct), _stream(stream)),
            "moesq_pack_weights")
+
+
+def moesq_import_dense_nvfp4(codes, scales, global_scale, e_begin: int, e_count: int, out: PackedWeights,
+                             stream=None):
+    _check(load().moesq_import_dense_nvfp4(_ptr(codes), _ptr(scales), _ptr(global_scale), e_begin, e_count,
+                                           ctypes.byref(out.struct), _stream(stream)), "moesq_import_dense_nvfp4")
+
+
+def moesq_export_dense_nvfp4(w: PackedWeights, codes, stream=None):
+    _check(load().moesq_export_dense_nvfp4(ctypes.byref(w.struct), _ptr(codes), _stream(stream)),
+           "moesq_export_dense_nvfp4")
 
 
 def moesq_route_permute(logits, rt: RoutingBuffers, stream=None):

@@ -20,7 +20,7 @@ namespace moesq {
 enum DevErrKind : int { kErrTimeout = 4, kErrFault = 5 };
 enum DevErrWhere : int {
   kWhereGemmProducer = 1, kWhereGemmMma = 2, kWhereGemmEpilogue = 3, kWhereGemmCounts = 4,
-  kWhereRoute = 5, kWhereQuant = 6, kWhereDebug = 7, kWhereSwiglu = 8, kWhereCombine = 9
+  kWhereRoute = 5, kWhereQuant = 6, kWhereDebug = 7, kWhereSwiglu = 8, kWhereCombine = 9, kWhereConvert = 10
 };
 
 __device__ int g_error_word;   // 0 = no error; (where << 8) | kind

@@ -408,6 +408,29 @@ moesq_status moesq_pack_weights(const uint16_t* w_bf16, int e_begin, int e_count
   return last_launch();
 }
 
+moesq_status moesq_import_dense_nvfp4(const uint8_t* codes, const uint8_t* scales, const float* global_scale,
+                                      int e_begin, int e_count, const moesq_weights* out, void* stream) {
+  MOESQ_TRY(check_weights(out));
+  if (!codes || !scales || !global_scale || !aligned(codes, 16)) return MOESQ_ERR_INVALID_ARG;
+  if (e_begin < 0 || e_count < 1 || e_begin + e_count > out->E) return MOESQ_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  const int M = out->M, K = out->K;
+  PackOut po{out->values, out->mask, out->scales, out->global_scale, out->ktiles};
+  const int64_t n_blocks = (int64_t)e_count * M * (K / 32);
+  import_dense_kernel<<<grid_for(n_blocks, 256, device_info().sms), 256, 0, s>>>(
+      codes, scales, global_scale, e_begin, n_blocks, M, K, po, out->global_scale);
+  return last_launch();
+}
+
+moesq_status moesq_export_dense_nvfp4(const moesq_weights* w, uint8_t* codes, void* stream) {
+  MOESQ_TRY(check_weights(w));
+  if (!codes || !aligned(codes, 16)) return MOESQ_ERR_INVALID_ARG;
+  const int64_t n_blocks = (int64_t)w->E * w->M * (w->K / 32);
+  export_dense_kernel<<<grid_for(n_blocks, 256, device_info().sms), 256, 0, as_stream(stream)>>>(
+      w->values, w->mask, n_blocks, w->K, codes);
+  return last_launch();
+}
+
 int64_t moesq_rows_capacity(int T, int k, int E) {
   if (T < 0 || k < 0 || E < 0) return 0;
   const int64_t R = (int64_t)T * k;

@@ -78,17 +78,46 @@ struct PackOut {
   uint8_t* ktiles;    // [E][M/128][K/256][kKTileBytes]
 };
 
+// Writes one 32-element block of an expert linear's packed form: the 8 code
+// bytes (the two kept pairs of each of its 4 groups, in K order), the 4 pair
+// bitmasks and the scale code, in the storage form and in the kernel-form
+// tile (swizzled values, metadata nibbles i0 | i1 << 2 of the two kept pair
+// indices, scales in the MMA layout).
+__device__ __forceinline__ void store_block(const PackOut& out, int e, int m, int b, int M, int K, uint2 vbytes,
+                                            const uint32_t (&bits4)[4], uint32_t code) {
+  const int nb_row = K / 32, KT = K / 256, MB = M / 128;
+  const int64_t row = (int64_t)e * M + m;
+  *reinterpret_cast<uint2*>(out.values + row * (K / 4) + (int64_t)b * 8) = vbytes;
+  const uint16_t mk = (uint16_t)(bits4[0] | (bits4[1] << 4) | (bits4[2] << 8) | (bits4[3] << 12));
+  *reinterpret_cast<uint16_t*>(out.mask + row * (K / 16) + (int64_t)b * 2) = mk;
+  out.scales[row * nb_row + b] = (uint8_t)code;
+  uint32_t meta = 0;
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    const uint32_t bits = bits4[g];
+    const uint32_t i0 = __ffs(bits) - 1;
+    const uint32_t i1 = 31 - __clz(bits);
+    meta |= (i0 | (i1 << 2)) << (4 * g);
+  }
+  const int mb = m >> 7, r = m & 127;
+  const int kt = b >> 3, bt = b & 7;            // 32-block within the 256-wide K tile
+  uint8_t* tile = out.ktiles + (((int64_t)e * MB + mb) * KT + kt) * kKTileBytes;
+  const int chunk = (bt >> 1) ^ ((r >> 1) & 3);  // 16-byte chunk after the swizzle
+  *reinterpret_cast<uint2*>(tile + r * 64 + chunk * 16 + (bt & 1) * 8) = vbytes;
+  *reinterpret_cast<uint16_t*>(tile + kKTileMeta + r * 16 + bt * 2) = (uint16_t)meta;
+  tile[kKTileScales + (bt >> 2) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (bt & 3)] = (uint8_t)code;
+}
+
 // Pass 2: one thread per 32-element block (4 groups, 16 kept values).
 __global__ void pack_blocks_kernel(const uint16_t* __restrict__ w, int e_begin, int64_t n_blocks, int M,
                                    int K, PackOut out) {
-  const int nb_row = K / 32, KT = K / 256, MB = M / 128;
+  const int nb_row = K / 32;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < n_blocks; t += stride) {
     const int b = (int)(t % nb_row);
     const int64_t row_local = t / nb_row;          // e_local * M + m
     const int e = e_begin + (int)(row_local / M);
     const int m = (int)(row_local % M);
-    const int64_t row = (int64_t)e * M + m;        // row of the full stack
     const uint16_t* src = w + row_local * K + (int64_t)b * 32;
 
     float kept[16];                                 // kept values of the block, K order
@@ -123,29 +152,77 @@ __global__ void pack_blocks_kernel(const uint16_t* __restrict__ w, int e_begin, 
     vbytes.x = quant8(h0, s_b, code == 0);
     vbytes.y = quant8(h1, s_b, code == 0);
 
-    // storage form
-    *reinterpret_cast<uint2*>(out.values + row * (K / 4) + (int64_t)b * 8) = vbytes;
-    const uint16_t mk = (uint16_t)(bits4[0] | (bits4[1] << 4) | (bits4[2] << 8) | (bits4[3] << 12));
-    *reinterpret_cast<uint16_t*>(out.mask + row * (K / 16) + (int64_t)b * 2) = mk;
-    out.scales[row * nb_row + b] = (uint8_t)code;
+    store_block(out, e, m, b, M, K, vbytes, bits4, code);
+  }
+}
 
-    // kernel form, tile (e, mb, kt): swizzled values, metadata nibbles
-    // i0 | i1 << 2 of the two kept pair indices, scales in the MMA layout
-    uint32_t meta = 0;
+// Dense NVFP4 codes of a tensor in the paired pattern -> pair-bitmask storage
+// and kernel form (model card, pair-bitmask v1): per 4-byte chunk the nonzero
+// bytes are kept; a chunk with fewer than 2 nonzero bytes keeps its
+// lowest-index zero bytes as well.  A chunk with more than 2 nonzero bytes is
+// not in the pattern: the device error word is set and its lowest two
+// nonzero bytes are kept.  One thread per 32-element block.
+__global__ void import_dense_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                                    const float* __restrict__ gamma_in, int e_begin, int64_t n_blocks, int M, int K,
+                                    PackOut out, float* __restrict__ gamma_out) {
+  const int nb_row = K / 32;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < n_blocks; t += stride) {
+    const int b = (int)(t % nb_row);
+    const int64_t row_local = t / nb_row;
+    const int e_local = (int)(row_local / M);
+    const int m = (int)(row_local % M);
+    const uint4 raw = *reinterpret_cast<const uint4*>(codes + row_local * (K / 2) + (int64_t)b * 16);
+    const uint32_t words[4] = {raw.x, raw.y, raw.z, raw.w};
+    uint32_t bits4[4], kept2[4];
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
-      const uint32_t bits = bits4[g];
-      const uint32_t i0 = __ffs(bits) - 1;
-      const uint32_t i1 = 31 - __clz(bits);
-      meta |= (i0 | (i1 << 2)) << (4 * g);
+      const uint32_t w = words[g];
+      uint32_t nz = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) nz |= ((w >> (8 * i)) & 0xFFu) != 0u ? (1u << i) : 0u;
+      if (__popc(nz) > 2) {                    // not in the pattern: keep the lowest two
+        record_error(kWhereConvert, kErrFault);
+        const uint32_t lo = nz & (0u - nz);
+        const uint32_t rest = nz & ~lo;
+        nz = lo | (rest & (0u - rest));
+      }
+      // fewer than two nonzero bytes: add the lowest-index zero bytes
+      if (__popc(nz) < 2) nz |= ~nz & (nz + 1u);
+      if (__popc(nz) < 2) nz |= ~nz & (nz + 1u);
+      bits4[g] = nz;
+      const uint32_t i0 = __ffs(nz) - 1, i1 = 31 - __clz(nz);
+      kept2[g] = ((w >> (8 * i0)) & 0xFFu) | (((w >> (8 * i1)) & 0xFFu) << 8);
     }
-    const int mb = m >> 7, r = m & 127;
-    const int kt = b >> 3, bt = b & 7;            // 32-block within the 256-wide K tile
-    uint8_t* tile = out.ktiles + (((int64_t)e * MB + mb) * KT + kt) * kKTileBytes;
-    const int chunk = (bt >> 1) ^ ((r >> 1) & 3);  // 16-byte chunk after the swizzle
-    *reinterpret_cast<uint2*>(tile + r * 64 + chunk * 16 + (bt & 1) * 8) = vbytes;
-    *reinterpret_cast<uint16_t*>(tile + kKTileMeta + r * 16 + bt * 2) = (uint16_t)meta;
-    tile[kKTileScales + (bt >> 2) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (bt & 3)] = (uint8_t)code;
+    const uint2 vbytes = make_uint2(kept2[0] | (kept2[1] << 16), kept2[2] | (kept2[3] << 16));
+    const uint32_t code = scales[row_local * nb_row + b];
+    store_block(out, e_begin + e_local, m, b, M, K, vbytes, bits4, code);
+    if (m == 0 && b == 0) gamma_out[e_begin + e_local] = gamma_in[e_local];
+  }
+}
+
+// Pair-bitmask storage form -> dense NVFP4 codes [E][M][K/2] (the kept bytes
+// at their chunk positions, zeros elsewhere).  One thread per 32-element block.
+__global__ void export_dense_kernel(const uint8_t* __restrict__ values, const uint8_t* __restrict__ mask,
+                                    int64_t n_blocks, int K, uint8_t* __restrict__ codes) {
+  const int nb_row = K / 32;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < n_blocks; t += stride) {
+    const int b = (int)(t % nb_row);
+    const int64_t row = t / nb_row;
+    const uint2 v = *reinterpret_cast<const uint2*>(values + row * (K / 4) + (int64_t)b * 8);
+    const uint32_t mk = *reinterpret_cast<const uint16_t*>(mask + row * (K / 16) + (int64_t)b * 2);
+    const uint32_t kept2[4] = {v.x & 0xFFFFu, v.x >> 16, v.y & 0xFFFFu, v.y >> 16};
+    uint32_t words[4];
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      const uint32_t nz = (mk >> (4 * g)) & 0xFu;
+      if (__popc(nz) != 2) record_error(kWhereConvert, kErrFault);
+      const uint32_t i0 = nz ? __ffs(nz) - 1 : 0, i1 = nz ? 31 - __clz(nz) : 1;
+      words[g] = ((kept2[g] & 0xFFu) << (8 * i0)) | ((kept2[g] >> 8) << (8 * i1));
+    }
+    *reinterpret_cast<uint4*>(codes + row * (K / 2) + (int64_t)b * 16) = make_uint4(words[0], words[1], words[2],
+                                                                                   words[3]);
   }
 }
 

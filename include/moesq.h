@@ -63,7 +63,9 @@ const char* moesq_last_cuda_error(void);
 
 /* Synchronises `stream`, then reads and clears the device error word.
  * *device_code (host) receives the raw word: 0 = none; otherwise
- * (where << 8) | kind, kind 4 = wait timeout, 5 = validation fault.
+ * (where << 8) | kind, kind 4 = wait timeout, 5 = validation fault;
+ * where: 1-4 grouped GEMM, 5 routing, 6 activation quantisation, 8 SwiGLU,
+ * 9 combine, 10 dense import / export.
  * Returns MOESQ_OK, MOESQ_ERR_TIMEOUT or MOESQ_ERR_DEVICE_FAULT. */
 moesq_status moesq_get_device_error(void* stream, int32_t* device_code);
 
@@ -131,6 +133,29 @@ size_t moesq_weights_bytes(int E, int M, int K, size_t* per_tensor);
  * out->global_scale of the packed experts is used as scratch first. */
 moesq_status moesq_pack_weights(const uint16_t* w_bf16, int e_begin, int e_count,
                                 const moesq_weights* out, void* stream);
+
+/* moesq_import_dense_nvfp4: weights already quantised to NVFP4 in the
+ * paired 4:8 pattern, held densely, -> the storage and kernel forms of `out`
+ * for experts [e_begin, e_begin + e_count) (model card "Kimi-K2.5-P48NVFP4-
+ * MoESQ", pair-bitmask v1 layout).  Inputs (device, e_count experts
+ * contiguous): codes [e_count][M][K/2] (two E2M1 codes per byte, even K in the
+ * low nibble), scales [e_count][M][K/32] (UE4M3, one per 32 dense K,
+ * row-major), global_scale [e_count] (the stored gamma).  Per 4-byte chunk
+ * (4 pairs of K) the nonzero bytes are kept; a chunk with fewer than two
+ * nonzero bytes keeps its lowest-index zero bytes as well (the model card's
+ * canonical rule), so dense -> pair-bitmask -> dense is lossless.  A chunk
+ * with more than two nonzero bytes is not in the pattern: the device error
+ * word gets a validation fault (where 10) and the chunk keeps its lowest two
+ * nonzero bytes.  codes must be 16-byte aligned. */
+moesq_status moesq_import_dense_nvfp4(const uint8_t* codes, const uint8_t* scales, const float* global_scale,
+                                      int e_begin, int e_count, const moesq_weights* out, void* stream);
+
+/* moesq_export_dense_nvfp4: the storage form of all w->E experts -> dense
+ * NVFP4 codes [E][M][K/2] (kept bytes at their chunk positions, zeros
+ * elsewhere); the scales and global scales of the dense form are w->scales
+ * and w->global_scale unchanged.  A mask nibble without exactly two bits set
+ * sets a validation fault (where 10).  codes must be 16-byte aligned. */
+moesq_status moesq_export_dense_nvfp4(const moesq_weights* w, uint8_t* codes, void* stream);
 
 /* ------------------------------------------------------------------ routing
  * Router output for T tokens, top-k of E experts.  Rows of every activation

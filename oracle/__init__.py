@@ -5,10 +5,11 @@ baseline of ``bench.py`` may import this package; the library and its Python
 binding never do.
 
 The arithmetic lives in plain C (``moesq_oracle.c``, built with gcc into
-``liboracle.so`` next to it); this module only marshals numpy arrays and
-composes the C steps into the MoE layer in the order the paper gives
-(arXiv 2610.02241, Sec. 3.4 and App. D.1).  Every C function cites its
-passage.  Parity status of each part is stated in the design doc.
+``liboracle.so`` next to it); this module marshals numpy arrays, composes
+the C steps into the MoE layer in the order the paper gives (arXiv
+2610.02241, Sec. 3.4 and App. D.1), and holds the two byte-layout converters
+between dense NVFP4 codes and the pair-bitmask form (integer rearrangement
+only, in numpy).  Every C function cites its passage.
 """
 from __future__ import annotations
 
@@ -147,6 +148,49 @@ def unpack_weights(values, mask, scales, gamma, M, K) -> np.ndarray:
     lib().oracle_unpack_weights(np.ascontiguousarray(values), np.ascontiguousarray(mask),
                                 np.ascontiguousarray(scales), float(gamma), M, K, out)
     return out
+
+
+def dense_from_sparse(values: np.ndarray, mask: np.ndarray) -> np.ndarray:
+    """Pair-bitmask storage -> dense NVFP4 codes (model card
+    "Kimi-K2.5-P48NVFP4-MoESQ", pair-bitmask v1): values [..., K/4] hold the 2
+    kept bytes of every 4-byte chunk in K order, mask [..., K/16] one nibble
+    per chunk (bit i = byte i kept, low nibble = lower-K chunk).  The kept
+    bytes go to the positions their nibble marks, zeros elsewhere."""
+    v = np.ascontiguousarray(values, dtype=np.uint8)
+    m = np.ascontiguousarray(mask, dtype=np.uint8)
+    lead = v.shape[:-1]
+    G = v.shape[-1] // 2                                   # 4-byte chunks per row
+    nib = np.stack([m & 15, m >> 4], axis=-1).reshape(lead + (G,)).astype(np.int64)
+    kept = v.reshape(lead + (G, 2))
+    lowest = np.array([(n & -n).bit_length() - 1 if n else 0 for n in range(16)])
+    highest = np.array([n.bit_length() - 1 if n else 1 for n in range(16)])
+    dense = np.zeros(lead + (G, 4), np.uint8)
+    np.put_along_axis(dense, lowest[nib][..., None], kept[..., 0:1], axis=-1)
+    np.put_along_axis(dense, highest[nib][..., None], kept[..., 1:2], axis=-1)
+    return dense.reshape(lead + (4 * G,))
+
+
+def sparse_from_dense(dense: np.ndarray):
+    """Dense NVFP4 codes [..., K/2] of a tensor in the paired pattern ->
+    (values [..., K/4], mask [..., K/16]) by the model card's canonical rule:
+    per 4-byte chunk the nonzero bytes are kept; with fewer than 2, its
+    lowest-index zero bytes are kept too.  Chunks with more than 2 nonzero
+    bytes are outside the pattern (ValueError)."""
+    d = np.ascontiguousarray(dense, dtype=np.uint8)
+    lead = d.shape[:-1]
+    G = d.shape[-1] // 4
+    ch = d.reshape(lead + (G, 4))
+    nz = ch != 0
+    cnt = nz.sum(-1)
+    if (cnt > 2).any():
+        raise ValueError("a 4-byte chunk has more than two nonzero bytes")
+    zero_rank = np.cumsum(~nz, axis=-1) - 1                # order of each zero byte within its chunk
+    keep = nz | (~nz & (zero_rank < (2 - cnt)[..., None]))
+    pos = np.argsort(~keep, axis=-1, kind="stable")[..., :2]   # the two kept positions, ascending
+    values = np.take_along_axis(ch, pos, axis=-1).reshape(lead + (2 * G,))
+    nib = (keep * (1 << np.arange(4))).sum(-1).astype(np.uint8)   # [..., G]
+    mask = (nib[..., 0::2] | (nib[..., 1::2] << 4)).astype(np.uint8)
+    return values, mask
 
 
 # ---------------------------------------------------------------- activations

@@ -177,3 +177,30 @@ def test_pack_is_deterministic_and_expert_independent():
     b = O.pack_weights(w[1:2])
     assert (a.values[1] == b.values[0]).all() and (a.mask[1] == b.mask[0]).all()
     assert (a.scales[1] == b.scales[0]).all() and a.gamma[1] == b.gamma[0]
+
+
+def test_oracle_converters_match_the_chunk_loops(packed):
+    """oracle.dense_from_sparse / sparse_from_dense (vectorised) against the
+    chunk-by-chunk restatement above, including chunks left with 0 or 1
+    nonzero bytes (the canonical rule's lowest-index zero bytes)."""
+    _, pk = packed
+    for e in range(pk.E):
+        dense = _dense_codes(pk, e)
+        assert (O.dense_from_sparse(pk.values[e], pk.mask[e]) == dense).all()
+        d = dense.copy()
+        d[:, 0:4] = 0                        # an empty chunk
+        d[:, 4:8] = 0
+        d[:, 6] = 0x31                       # a chunk with one nonzero byte
+        v_loop, m_loop = _sparse_from_dense(d)
+        v, m = O.sparse_from_dense(d)
+        assert (v == v_loop).all() and (m == m_loop).all()
+        assert (O.dense_from_sparse(v, m) == d).all()
+        nib = np.stack([m & 15, m >> 4], -1)
+        assert (np.vectorize(lambda x: bin(int(x)).count("1"))(nib) == 2).all()
+
+
+def test_oracle_sparse_from_dense_rejects_three_nonzero_bytes():
+    d = np.zeros((1, 8), np.uint8)
+    d[0, :3] = 0x11
+    with pytest.raises(ValueError):
+        O.sparse_from_dense(d)
