@@ -113,11 +113,13 @@ def outlier_channels(key: int, K: int, count: int = 4) -> np.ndarray:
 
 
 def activations_bf16_np(seed: int, T: int, K: int, n_outliers: int = 4,
-                        outlier_gain: float = 20.0, label: int = 0) -> np.ndarray:
+                        outlier_gain: float = 20.0, label: int = 0, rows: int = None) -> np.ndarray:
     """Hidden states X [T, K] ~ N(0, 1) with `n_outliers` channels scaled by
-    `outlier_gain`, as bf16 bit patterns."""
+    `outlier_gain`, as bf16 bit patterns.  rows < T draws only the first
+    `rows` rows (the same values as the first rows of the full batch)."""
     key = stream_key(seed, 1, label)
-    v = normal_f64_np(key, 0, T * K).reshape(T, K)
+    n = T if rows is None else min(rows, T)
+    v = normal_f64_np(key, 0, n * K).reshape(n, K)
     if n_outliers:
         ch = outlier_channels(stream_key(seed, 2, label), K, n_outliers)
         v[:, ch] *= outlier_gain
