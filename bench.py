@@ -284,8 +284,14 @@ def run_cuda(args, rank, world, local_rank):
         m.moesq_route_permute(lg, rb)
         m.moesq_quantize_act(x, T, K_in, rb, ga, rb.rows_cap, a_codes, a_scales)
 
+    # GEMM configurations, frozen by moesq_gemm_autotune after the warm-up
+    # and before the graphs are captured
+    tuned = {"main": (0, 0), "down": (0, 0)}
+
     def c_gemm_main():
-        m.moesq_grouped_sparse_gemm(w_main, a_codes, a_scales, rb.rows_cap, rb.counts, rb.row_offsets, ga, y_main)
+        tn, nc = tuned["main"]
+        m.moesq_grouped_sparse_gemm(w_main, a_codes, a_scales, rb.rows_cap, rb.counts, rb.row_offsets, ga, y_main,
+                                    tile_n=tn, num_ctas=nc)
 
     if kind == "quant_gemm":                  # fixed grouping: routed once, outside the step
         m.moesq_route_permute(lg, rb)
@@ -296,7 +302,8 @@ def run_cuda(args, rank, world, local_rank):
     if kind == "layer":
         comps += [("swiglu_quant", lambda: m.moesq_swiglu_quant(y_main, I, rb, gh, h_codes, h_scales)),
                   ("gemm_down", lambda: m.moesq_grouped_sparse_gemm(w_dn, h_codes, h_scales, rb.rows_cap, rb.counts,
-                                                                    rb.row_offsets, gh, y_dn)),
+                                                                    rb.row_offsets, gh, y_dn, tile_n=tuned["down"][0],
+                                                                    num_ctas=tuned["down"][1])),
                   ("combine", lambda: m.moesq_combine(y_dn, H, rb, out))]
 
     def step_eager():
@@ -313,6 +320,13 @@ def run_cuda(args, rank, world, local_rank):
     st, word = m.moesq_get_device_error()
     if st != 0:
         raise RuntimeError("device error word %#x during warm-up" % word)
+    tuned["main"] = m.moesq_gemm_autotune(w_main, a_codes, a_scales, rb.rows_cap, rb.counts, rb.row_offsets, ga,
+                                          y_main, reps=3)[0]
+    if kind == "layer":
+        tuned["down"] = m.moesq_gemm_autotune(w_dn, h_codes, h_scales, rb.rows_cap, rb.counts, rb.row_offsets, gh,
+                                              y_dn, reps=3)[0]
+    step_eager()                              # outputs of the tuned configuration
+    torch.cuda.synchronize()
     counts = rb.counts.cpu().numpy()
 
     # One CUDA graph per step (the pages time CUDA-graph replays, App. D.2),
@@ -408,7 +422,7 @@ def run_cuda(args, rank, world, local_rank):
     if e2e:
         e2e["ms_per_step"] = e2e_max
     return dict(kind=kind, E=E, k=k, H=H, I=I, T=T, routing=routing, ms=t_max, parts=parts, flops=flops,
-                wbytes=wbytes, gemm_bytes=gemm_bytes, gemm_fl=gemm_fl, e2e=e2e, clocks=clk, launches=launches_per_step * args.steps,
+                wbytes=wbytes, gemm_bytes=gemm_bytes, gemm_fl=gemm_fl, e2e=e2e, tuned=tuned, clocks=clk, launches=launches_per_step * args.steps,
                 wall_s=t_wall, counts=counts)
 
 
@@ -585,6 +599,8 @@ def main():
             "vs_baseline": vs_baseline, "dtype": "nvfp4 (e2m1 x ue4m3 products, f32 accumulate, bf16 out)",
             "data": "synthetic (seeded; pages' shapes and distributions)", "config": config,
             "weight_gbs": weight_gbs, "breakdown_ms": r["parts"], "roofline": roofline,
+            "gemm_config": {name: {"tile_n": tn, "num_ctas": nc} for name, (tn, nc) in r["tuned"].items()
+                            if tn},
             "clocks": r["clocks"], "gpu_launches": r["launches"],
             "expert_rows": {"min": int(r["counts"].min()), "max": int(r["counts"].max()),
                             "touched": int((r["counts"] > 0).sum())}}

@@ -67,6 +67,8 @@ def load():
         "moesq_set_wait_timeout_ns": (None, [_c.c_uint64]),
         "moesq_weights_bytes": (_sz, [_c.c_int, _c.c_int, _c.c_int, _P(_sz)]),
         "moesq_pack_weights": (_c.c_int, [_vp, _c.c_int, _c.c_int, _P(moesq_weights), _vp]),
+        "moesq_gemm_autotune": (_c.c_int, [_P(moesq_weights), _vp, _vp, _c.c_int, _vp, _vp, _vp, _vp, _c.c_int,
+                                           _P(moesq_gemm_config), _P(_c.c_float), _vp]),
         "moesq_import_dense_nvfp4": (_c.c_int, [_vp, _vp, _vp, _c.c_int, _c.c_int, _P(moesq_weights), _vp]),
         "moesq_export_dense_nvfp4": (_c.c_int, [_P(moesq_weights), _vp, _vp]),
         "moesq_rows_capacity": (_i64, [_c.c_int, _c.c_int, _c.c_int]),
@@ -208,6 +210,17 @@ def moesq_layer_host_workspace_bytes(T: int, k: int, E: int, H: int, I: int) -> 
 def moesq_pack_weights(w_bf16, e_begin: int, e_count: int, out: PackedWeights, stream=None):
     _check(load().moesq_pack_weights(_ptr(w_bf16), e_begin, e_count, ctypes.byref(out.struct), _stream(stream)),
            "moesq_pack_weights")
+
+
+def moesq_gemm_autotune(w: PackedWeights, a_codes, a_scales, rows_cap: int, counts, row_offsets, gamma_a, y_bf16,
+                        reps: int = 5, stream=None):
+    """Fastest (tile_n, num_ctas) for these inputs and its mean time in ms."""
+    cfg = moesq_gemm_config(0, 0)
+    ms = _c.c_float(0.0)
+    _check(load().moesq_gemm_autotune(ctypes.byref(w.struct), _ptr(a_codes), _ptr(a_scales), rows_cap, _ptr(counts),
+                                      _ptr(row_offsets), _ptr(gamma_a), _ptr(y_bf16), reps, ctypes.byref(cfg),
+                                      ctypes.byref(ms), _stream(stream)), "moesq_gemm_autotune")
+    return (cfg.tile_n, cfg.num_ctas), ms.value
 
 
 def moesq_import_dense_nvfp4(codes, scales, global_scale, e_begin: int, e_count: int, out: PackedWeights,

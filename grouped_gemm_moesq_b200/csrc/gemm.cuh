@@ -157,7 +157,9 @@ grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const GemmP
   int local_bad = 0;
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     const int c = p.counts[e], r0 = p.row_offsets[e], r1 = p.row_offsets[e + 1];
-    const bool ok = c >= 0 && r0 >= 0 && (r0 & 127) == 0 && r1 - r0 == ((c + 127) & ~127) && r1 <= p.rows_cap;
+    // each expert's span starts on a 128-row boundary and holds its rows
+    // (padded to 128); spans may leave gaps, e.g. a fixed capacity per expert
+    const bool ok = c >= 0 && r0 >= 0 && (r0 & 127) == 0 && r1 - r0 >= ((c + 127) & ~127) && r1 <= p.rows_cap;
     local_bad |= ok ? 0 : 1;
     cnt[e] = ok ? c : 0;
     rstart[e] = r0;

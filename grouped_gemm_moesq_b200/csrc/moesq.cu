@@ -511,6 +511,47 @@ moesq_status moesq_grouped_sparse_gemm(const moesq_weights* w, const uint8_t* a_
   return launch_gemm<128>(w, a_codes, a_scales, rows_cap, counts, row_offsets, gamma_a, y_bf16, num_ctas, s);
 }
 
+moesq_status moesq_gemm_autotune(const moesq_weights* w, const uint8_t* a_codes, const uint8_t* a_scales,
+                                 int rows_cap, const int32_t* counts, const int32_t* row_offsets,
+                                 const float* gamma_a, uint16_t* y_bf16, int reps,
+                                 moesq_gemm_config* best, float* best_ms, void* stream) {
+  if (!best || !best_ms || reps < 1) return MOESQ_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  const int sms = device_info().sms;
+  const moesq_gemm_config cands[4] = {{64, 2 * sms}, {128, 2 * sms}, {64, sms}, {128, sms}};
+  cudaEvent_t ev[2];
+  MOESQ_CUDA(cudaEventCreate(&ev[0]));
+  if (cudaEventCreate(&ev[1]) != cudaSuccess) {
+    cudaEventDestroy(ev[0]);
+    return MOESQ_ERR_CUDA;
+  }
+  moesq_status st = MOESQ_OK;
+  float best_t = -1.0f;
+  for (const moesq_gemm_config& c : cands) {
+    st = moesq_grouped_sparse_gemm(w, a_codes, a_scales, rows_cap, counts, row_offsets, gamma_a, y_bf16, &c, s);
+    if (st != MOESQ_OK) break;
+    if (cudaEventRecord(ev[0], s) != cudaSuccess) { st = MOESQ_ERR_CUDA; break; }
+    for (int r = 0; r < reps && st == MOESQ_OK; ++r)
+      st = moesq_grouped_sparse_gemm(w, a_codes, a_scales, rows_cap, counts, row_offsets, gamma_a, y_bf16, &c, s);
+    if (st != MOESQ_OK) break;
+    float ms = 0.0f;
+    if (cudaEventRecord(ev[1], s) != cudaSuccess || cudaEventSynchronize(ev[1]) != cudaSuccess ||
+        cudaEventElapsedTime(&ms, ev[0], ev[1]) != cudaSuccess) {
+      st = MOESQ_ERR_CUDA;
+      break;
+    }
+    ms /= (float)reps;
+    if (best_t < 0.0f || ms < best_t) {
+      best_t = ms;
+      *best = c;
+    }
+  }
+  cudaEventDestroy(ev[0]);
+  cudaEventDestroy(ev[1]);
+  if (st == MOESQ_OK) *best_ms = best_t;
+  return st;
+}
+
 moesq_status moesq_swiglu_quant(const uint16_t* y_gu, int I, const moesq_routing* rt, const float* gamma_h,
                                 uint8_t* h_codes, uint8_t* h_scales, void* stream) {
   MOESQ_TRY(check_routing(rt));

@@ -253,8 +253,14 @@ moesq_status moesq_act_global_scale(const uint16_t* x_bf16, int64_t n, float* ga
  * W_e X_e^T with the weight as the sparse operand, both block scales applied
  * in the MMA, the tensor scales folded into alpha_e in the epilogue).
  * a_codes [rows_cap][K/2], a_scales in the MMA scale layout, y [rows_cap][M]
- * bf16 (only valid rows are written).  counts [E], row_offsets [E+1] as in
- * moesq_routing (device); they are validated on the device.
+ * bf16 (only valid rows are written).  counts [E] and row_offsets [E+1]
+ * (device) give expert e the rows row_offsets[e] + [0, counts[e]); each
+ * row_offsets[e] is a multiple of 128 and each span row_offsets[e+1] -
+ * row_offsets[e] holds at least counts[e] rounded up to 128, so both the
+ * compact aligned layout of moesq_routing and a fixed capacity N per expert
+ * (row_offsets[e] = e * N, N a multiple of 128: the paper's App. D.1
+ * batched layout) qualify.  They are validated on the device (validation
+ * fault, where 4, and no output otherwise).
  * cfg may be NULL (defaults).                                            */
 typedef struct {
   int32_t tile_n;      /* token rows per tile: 0 = auto, 64 or 128 */
@@ -267,6 +273,19 @@ moesq_status moesq_grouped_sparse_gemm(const moesq_weights* w, const uint8_t* a_
                                        const int32_t* counts, const int32_t* row_offsets,
                                        const float* gamma_a, uint16_t* y_bf16,
                                        const moesq_gemm_config* cfg, void* stream);
+
+/* moesq_gemm_autotune: times moesq_grouped_sparse_gemm on these inputs for
+ * each candidate configuration (token tile 64 or 128 rows, x one or two
+ * persistent CTAs per SM), one warm-up launch and `reps` timed launches each
+ * (CUDA events on `stream`), and writes the fastest to *best and its mean
+ * time in milliseconds to *best_ms (the paper freezes one kernel variant
+ * per problem geometry before CUDA-graph capture, App. D.1).  Writes y_bf16
+ * as the GEMM does; synchronises the stream, so call it before a capture.
+ * reps >= 1. */
+moesq_status moesq_gemm_autotune(const moesq_weights* w, const uint8_t* a_codes, const uint8_t* a_scales,
+                                 int rows_cap, const int32_t* counts, const int32_t* row_offsets,
+                                 const float* gamma_a, uint16_t* y_bf16, int reps,
+                                 moesq_gemm_config* best, float* best_ms, void* stream);
 
 /* ------------------------------------------------------------- layer parts
  * moesq_swiglu_quant: h = SiLU(g) * u for every valid row of the gate_up

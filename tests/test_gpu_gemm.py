@@ -171,3 +171,65 @@ def test_gemm_rejects_inconsistent_counts(cuda_lib):
     assert float(y.float().abs().max()) == 0.0
     ok, info = _run_isolated(m, pk, np.array([3, 4]), K, 10, 0)
     assert ok
+
+
+@pytest.mark.parametrize("tile_n", [64, 128])
+def test_gemm_fixed_capacity_layout(cuda_lib, tile_n):
+    """The paper's batched layout (App. D.1): expert e's rows start at e * N
+    for a fixed capacity N; the GEMM reads and writes those rows only."""
+    torch = pytest.importorskip("torch")
+    m = cuda_lib
+    E, M, K, cap = 5, 256, 512, 256
+    counts = np.array([3, 0, 130, 64, 1])
+    pk = O.pack_weights(weights_np(17, 0, E, M, K))
+    R = int(counts.sum())
+    x = S.activations_bf16_np(18, R, K)
+    ga = np.full(E, np.float32(O.act_global_scale(x)), np.float32)
+    offs = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    codes, scales = O.quantize_rows_bf16(x, ga[0])
+    y_ref, basis = O.grouped_gemm(pk, codes, scales, offs, ga)
+    rows = np.concatenate([e * cap + np.arange(counts[e]) for e in range(E)]).astype(np.int64)
+    rc = E * cap
+    c_rows = np.zeros((rc, K // 2), np.uint8)
+    s_rows = np.zeros((rc, K // 32), np.uint8)
+    c_rows[rows], s_rows[rows] = codes, scales
+    y = torch.full((rc, M), float("nan"), dtype=torch.bfloat16, device="cuda")
+    m.moesq_grouped_sparse_gemm(packed_from_oracle(m, pk), to_dev(c_rows), to_dev(L.scales_to_mma(s_rows)), rc,
+                                to_dev(counts.astype(np.int32)), to_dev((np.arange(E + 1) * cap).astype(np.int32)),
+                                to_dev(ga), y, tile_n=tile_n)
+    st, word = m.moesq_get_device_error()
+    assert st == 0, "device error word %#x" % word
+    yn = to_np(y)
+    ok, err, bound, bad = gemm_tolerance_ok(yn[rows], y_ref, basis)
+    assert ok, err.max()
+    untouched = np.setdiff1d(np.arange(rc), rows)
+    assert np.isnan(S.bf16_bits_to_f32_np(yn[untouched])).all()       # gaps are not written
+
+
+def test_gemm_autotune_picks_a_candidate_and_stays_correct(cuda_lib):
+    """moesq_gemm_autotune returns one of its candidate configurations with a
+    positive time, and the GEMM under that configuration matches the oracle."""
+    torch = pytest.importorskip("torch")
+    m = cuda_lib
+    E, M, K = 6, 256, 512
+    counts = np.array([5, 70, 0, 130, 1, 17])
+    pk = O.pack_weights(weights_np(23, 0, E, M, K))
+    R = int(counts.sum())
+    x = S.activations_bf16_np(24, R, K)
+    ga = np.full(E, np.float32(O.act_global_scale(x)), np.float32)
+    offs = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    codes, scales = O.quantize_rows_bf16(x, ga[0])
+    y_ref, basis = O.grouped_gemm(pk, codes, scales, offs, ga)
+    c_rows, s_mma, rc = act_rows_from_compact(codes, scales, counts, K)
+    pw = packed_from_oracle(m, pk)
+    args = (to_dev(c_rows), to_dev(s_mma), rc, to_dev(counts.astype(np.int32)), to_dev(L.aligned_rows(counts)),
+            to_dev(ga))
+    y = torch.zeros((rc, M), dtype=torch.bfloat16, device="cuda")
+    (tile_n, num_ctas), ms = m.moesq_gemm_autotune(pw, *args, y, reps=2)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert tile_n in (64, 128) and num_ctas in (sms, 2 * sms) and ms > 0
+    y.fill_(float("nan"))
+    m.moesq_grouped_sparse_gemm(pw, *args, y, tile_n=tile_n, num_ctas=num_ctas)
+    assert m.moesq_get_device_error()[0] == 0
+    ok, err, bound, bad = gemm_tolerance_ok(to_np(y)[L.compact_to_rows(counts)], y_ref, basis)
+    assert ok, err.max()
