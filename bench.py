@@ -108,6 +108,28 @@ def profiled_traffic(workload, gemm):
     return None
 
 
+def gemm_roofline(gbytes, gfl, gemm_ms, peaks, traffic, gname):
+    """Roofline of one grouped GEMM launch: the bound is whichever ideal time
+    is longer, algorithmic bytes at the HBM copy rate or dense-equivalent
+    flops at the sparse NVFP4 tensor rate; both fractions are reported."""
+    hbm_peak = peaks["hbm_gbs"]
+    tc_peak = peaks["bf16_tflops"] * FP4_OVER_BF16 * SPARSE_FACTOR
+    hbm_ach = gbytes / (gemm_ms * 1e-3) / 1e9
+    tc_ach = gfl / (gemm_ms * 1e-3) / 1e12
+    if gbytes / (hbm_peak * 1e9) >= gfl / (tc_peak * 1e12):
+        roofline = {"bound": "hbm", "achieved": hbm_ach, "peak": hbm_peak, "unit": "GB/s",
+                    "frac": hbm_ach / hbm_peak}
+    else:
+        roofline = {"bound": "tensor", "achieved": tc_ach, "peak": tc_peak, "unit": "TFLOP/s",
+                    "frac": tc_ach / tc_peak}
+    roofline.update({"traffic": traffic, "algorithmic_bytes": gbytes, "dense_equiv_flops": gfl,
+                     "kernel": "grouped_sparse_gemm (%s)" % gname, "kernel_ms": gemm_ms,
+                     "hbm_frac": hbm_ach / hbm_peak, "tensor_frac": tc_ach / tc_peak,
+                     "peak_source": "%s (tensor peak = dense bf16 burst x %g fp4/bf16 x %g sparse)"
+                     % (peaks["source"], FP4_OVER_BF16, SPARSE_FACTOR)})
+    return roofline
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -574,24 +596,7 @@ def main():
     gname = "down" if r["kind"] == "gemm_down" else "gate_up"
     gemm_ms = r["parts"]["gemm_main"]
     gbytes, gfl = r["gemm_bytes"][gname], r["gemm_fl"][gname]
-    # the bound is whichever ideal time is longer: algorithmic bytes at the HBM
-    # copy rate, or dense-equivalent flops at the sparse NVFP4 tensor rate
-    hbm_peak = peaks["hbm_gbs"]
-    tc_peak = peaks["bf16_tflops"] * FP4_OVER_BF16 * SPARSE_FACTOR
-    hbm_ach = gbytes / (gemm_ms * 1e-3) / 1e9
-    tc_ach = gfl / (gemm_ms * 1e-3) / 1e12
-    traffic = profiled_traffic(args.workload, gname)
-    if gbytes / (hbm_peak * 1e9) >= gfl / (tc_peak * 1e12):
-        roofline = {"bound": "hbm", "achieved": hbm_ach, "peak": hbm_peak, "unit": "GB/s",
-                    "frac": hbm_ach / hbm_peak}
-    else:
-        roofline = {"bound": "tensor", "achieved": tc_ach, "peak": tc_peak, "unit": "TFLOP/s",
-                    "frac": tc_ach / tc_peak}
-    roofline.update({"traffic": traffic, "algorithmic_bytes": gbytes, "dense_equiv_flops": gfl,
-                     "kernel": "grouped_sparse_gemm (%s)" % gname, "kernel_ms": gemm_ms,
-                     "hbm_frac": hbm_ach / hbm_peak, "tensor_frac": tc_ach / tc_peak,
-                     "peak_source": "%s (tensor peak = dense bf16 burst x %g fp4/bf16 x %g sparse)"
-                     % (peaks["source"], FP4_OVER_BF16, SPARSE_FACTOR)})
+    roofline = gemm_roofline(gbytes, gfl, gemm_ms, peaks, profiled_traffic(args.workload, gname), gname)
     tab11_n = T // 30 if args.workload.startswith("tab11_") else None
     vs_baseline = value / TAB11[tab11_n][1] if tab11_n else None
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,

@@ -74,3 +74,28 @@ def test_tab11_pattern_routes_to_the_paper_counts():
         rt = O.route(bench.tab11_logits(T, 384), 8)
         want = np.array([n * (4 - g % 4) // 4 for g in range(384)])
         assert (rt.counts == want).all()
+
+
+def test_gemm_roofline_picks_the_longer_ideal_time():
+    """Decode-like launch (bytes dominate) is HBM-bound, a launch with many
+    rows per expert is tensor-bound; fractions are achieved / peak."""
+    import bench
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1500.0, "source": "measured"}
+    r = bench.gemm_roofline(3.0e9, 1.0e11, 0.5, peaks, None, "gate_up")        # 0.5 ms
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert r["frac"] == pytest.approx(3.0e9 / 0.5e-3 / 1e9 / 6000.0)
+    tc_peak = 1500.0 * bench.FP4_OVER_BF16 * bench.SPARSE_FACTOR
+    r = bench.gemm_roofline(1.0e9, 2.0e15, 1.0, peaks, 123, "down")             # 1 ms
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s" and r["traffic"] == 123
+    assert r["frac"] == pytest.approx(2.0e15 / 1e-3 / 1e12 / tc_peak)
+    assert r["hbm_frac"] == pytest.approx(1.0e9 / 1e-3 / 1e9 / 6000.0)
+
+
+def test_traffic_record_needs_the_current_gemm_source():
+    """profiles/ records are only used while their source hash matches."""
+    import bench
+    sha = bench.gemm_source_sha()
+    t = bench.profiled_traffic("30b_layer_t256", "gate_up")
+    assert t is None or isinstance(t, int)
+    assert bench.profiled_traffic("no_such_workload", "gate_up") is None
+    assert len(sha) == 16
