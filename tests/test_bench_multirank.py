@@ -99,3 +99,34 @@ def test_traffic_record_needs_the_current_gemm_source():
     assert t is None or isinstance(t, int)
     assert bench.profiled_traffic("no_such_workload", "gate_up") is None
     assert len(sha) == 16
+
+
+def test_bench_line_has_the_contract_keys(monkeypatch, capsys):
+    """bench.main() composes one JSON line with every key of the contract
+    (a stand-in for the CUDA run supplies the measured parts)."""
+    import json
+    import sys
+    import bench
+    E, k, H, I, T, routing, kind = bench.WORKLOADS[bench.DEFAULT_WORKLOAD]
+    counts = np.full(E, T * k // E)
+    flops, wbytes, gbytes, gfl = bench.step_work(E, k, H, I, T, counts, kind)
+
+    def fake_run(args, rank, world, local_rank):
+        return dict(kind=kind, E=E, k=k, H=H, I=I, T=T, routing=routing, ms=0.08, parts={"gemm_main": 0.036},
+                    flops=flops, wbytes=wbytes, gemm_bytes=gbytes, gemm_fl=gfl,
+                    e2e={"ms_per_step": 0.16, "h2d_bytes_per_step": 1, "d2h_bytes_per_step": 2},
+                    tuned={"main": (64, 296), "down": (64, 296)},
+                    clocks={"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}, launches=140, wall_s=0.01,
+                    counts=counts)
+
+    monkeypatch.setattr(bench, "run_cuda", fake_run)
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--steps", "20", "--warmup", "3", "--no-cpu-baseline"])
+    bench.main()
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "clocks", "gpu_launches"):
+        assert key in line, key
+    assert line["config"]["workload"] == bench.DEFAULT_WORKLOAD
+    assert line["roofline"]["bound"] == "hbm" and 0 < line["roofline"]["frac"]
+    assert line["e2e"]["value"] > 0 and line["gpu_launches"] == 140
+    assert line["value"] == pytest.approx(flops / 0.08e-3 / 1e12)
