@@ -5,7 +5,9 @@
 // (paper App. A Eq. 6 pattern set; model card "exactly 2 pairs are kept").
 // Scales: paper Sec. 3.4 Eq. 5 on the masked weights; values: Eq. 3.
 // Outputs the storage form of the model card (values / mask / scales /
-// gamma) and the kernel form read by the grouped GEMM (ktiles).
+// gamma) and the kernel form read by the grouped GEMM (ktiles).  Also the
+// converters between dense NVFP4 codes and that storage form (the model
+// card's canonical rule for chunks with fewer than two nonzero bytes).
 #pragma once
 #include "common.cuh"
 

@@ -3,6 +3,9 @@
 // (expert, token, slot) permutation.  Integer outputs are exact and
 // independent of thread scheduling: ranks come from per-block token bitmaps
 // (atomicOr is order-free) and popcounts, never from atomic counters.
+// Kernels: route_topk_kernel (one warp per token), then either
+// route_finish_kernel (one CTA, T <= kRouteSmallMaxT) or route_count_kernel,
+// route_scan_kernel and route_scatter_kernel (blocks of kRouteTPB tokens).
 #pragma once
 #include "common.cuh"
 
