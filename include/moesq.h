@@ -15,7 +15,8 @@
  *    void*, NULL = the legacy default stream), does no host synchronisation
  *    and reads no device data on the host, so a sequence of calls can be
  *    captured into a CUDA graph.  The exceptions are moesq_get_device_error
- *    (synchronises) and moesq_moe_layer_host (synchronises at the end).
+ *    (synchronises), moesq_moe_layer_host (synchronises at the end) and
+ *    moesq_gemm_autotune (times launches, synchronises).
  *  - Shape and argument errors are detected on the host and returned at once;
  *    nothing is launched then.  Faults detected on the device (inconsistent
  *    routing counts, out-of-range expert ids, a bounded wait that ran out)
