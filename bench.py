@@ -27,6 +27,7 @@ import glob
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -86,12 +87,21 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
 
 
+def strip_c_comments(text):
+    """C/C++ source without comments and whitespace (string literals in
+    these sources hold no comment markers)."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return re.sub(r"\s+", "", text)
+
+
 def gemm_source_sha():
-    """Hash of the sources the grouped GEMM kernel is built from; a DRAM
-    traffic record taken with ncu is only used while it matches."""
+    """Hash of the code (comments and whitespace removed) of the sources the
+    grouped GEMM kernel is built from; a DRAM traffic record taken with ncu
+    is only used while it matches."""
     h = hashlib.sha256()
     for f in ("gemm.cuh", "common.cuh"):
-        h.update(open(os.path.join(ROOT, "grouped_gemm_moesq_b200", "csrc", f), "rb").read())
+        h.update(strip_c_comments(open(os.path.join(ROOT, "grouped_gemm_moesq_b200", "csrc", f)).read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -45,9 +45,9 @@ constexpr int kGemmThreads = 192;   // producer, MMA, 4 epilogue warps
 
 template <int TN>
 struct GemmCfg {
-  // Two CTAs share an SM: each is one copy -> MMA issue chain, and two
-  // independent chains keep the tensor pipe busier than one (a chain waits,
-  // per K step, for its copies to land before its MMAs can go).
+  // Two CTAs share an SM: each issues its tcgen05 copies and MMAs from one
+  // thread, and two such independent issue streams keep the tensor pipe
+  // busier than one.
   static constexpr int kCtasPerSm = 2;
   static constexpr int kNAcc = (TN == 128) ? 1 : 2;     // accumulator buffers (TN columns each)
   static constexpr int kStages = (TN == 128) ? 3 : 5;
