@@ -233,3 +233,51 @@ def test_gemm_autotune_picks_a_candidate_and_stays_correct(cuda_lib):
     assert m.moesq_get_device_error()[0] == 0
     ok, err, bound, bad = gemm_tolerance_ok(to_np(y)[L.compact_to_rows(counts)], y_ref, basis)
     assert ok, err.max()
+
+
+def _prefill_rows(n):
+    """Row indices checked in an expert with n rows: the first 32, 32 that
+    straddle a 128-row token-tile boundary, and the last tile's rows."""
+    idx = set(range(min(n, 32)))
+    if n > 160:
+        idx.update(range(112, 144))
+    last = (n - 1) // 128 * 128
+    idx.update(range(last, n))
+    return np.array(sorted(idx), np.int64)
+
+
+def test_gemm_kimi_prefill_down_full_size_sampled(cuda_lib):
+    """Kimi-shaped down projection at full size (E=384, M=7168, K=2048),
+    T=8192 with Zipf(1.1) routing, as the prefill bench runs it: sampled rows
+    of the heaviest expert (several token tiles, a partial last tile) and all
+    rows of the lightest, against the oracle."""
+    torch = pytest.importorskip("torch")
+    m = cuda_lib
+    E, M, K, T, k = 384, 7168, 2048, 8192, 8
+    pw = pack_gpu_generated(m, 31, 1, E, M, K, chunk=8)
+    x = S.activations_bf16_np(31, T, K)
+    lg = S.zipf_logits_np(1234, T, E)
+    rt = O.route(lg, k)
+    ga = np.full(E, O.act_global_scale(x), np.float32)
+    rb = m.RoutingBuffers(T, E, k)
+    m.moesq_route_permute(to_dev(lg), rb)
+    assert (to_np(rb.counts) == rt.counts).all()
+    codes, scales = m.act_buffers(rb.rows_cap, K)
+    m.moesq_quantize_act(to_dev(x), T, K, rb, to_dev(ga), rb.rows_cap, codes, scales)
+    y = torch.full((rb.rows_cap, M), float("nan"), dtype=torch.bfloat16, device="cuda")
+    m.moesq_grouped_sparse_gemm(pw, codes, scales, rb.rows_cap, rb.counts, rb.row_offsets, to_dev(ga), y)
+    assert m.moesq_get_device_error()[0] == 0
+    yg_all = to_np(y)
+    ro = L.aligned_rows(rt.counts)
+    used = np.nonzero(rt.counts)[0]
+    heavy, light = int(np.argmax(rt.counts)), int(used[np.argmin(rt.counts[used])])
+    for e in (heavy, light):
+        n = int(rt.counts[e])
+        idx = _prefill_rows(n) if e == heavy else np.arange(n)
+        pk = O.pack_weights(S.expert_weights_bf16_np(31, 1, e, M, K)[None])
+        s0 = rt.offsets[e]
+        toks = rt.sorted_to_slot[s0:s0 + n][idx] // k
+        c, s = O.quantize_rows_bf16(x[toks], ga[e])
+        y_ref, basis = O.grouped_gemm(pk, c, s, np.array([0, idx.size], np.int32), ga[e:e + 1])
+        ok, err, bound, bad = gemm_tolerance_ok(yg_all[ro[e] + idx], y_ref, basis)
+        assert ok, (e, n, err.max())
