@@ -75,6 +75,11 @@ def lib():
         L.oracle_grouped_gemm.restype = None
         L.oracle_grouped_gemm.argtypes = [_u8, _u8, _u8, _f32, _c.c_int, _c.c_int, _c.c_int,
                                           _u8, _u8, _i32, _f32, _u16, _c.c_void_p, _c.c_void_p]
+        L.oracle_pack_dense_nvfp4.restype = None
+        L.oracle_pack_dense_nvfp4.argtypes = [_u16, _c.c_int, _c.c_int, _u8, _u8, _f32]
+        L.oracle_dense_grouped_gemm.restype = None
+        L.oracle_dense_grouped_gemm.argtypes = [_u8, _u8, _f32, _c.c_int, _c.c_int, _c.c_int,
+                                                _u8, _u8, _i32, _f32, _u16, _c.c_void_p, _c.c_void_p]
         L.oracle_swiglu.restype = None
         L.oracle_swiglu.argtypes = [_u16, _c.c_int, _c.c_int, _f32]
         L.oracle_combine.restype = None
@@ -263,6 +268,47 @@ def grouped_gemm(pk: Packed, a_codes, a_scales, offsets, gamma_a, want_exact=Fal
                               np.ascontiguousarray(offsets, np.int32),
                               np.ascontiguousarray(gamma_a, np.float32), y,
                               exact.ctypes.data if want_exact else None, basis.ctypes.data)
+    return (y, basis, exact) if want_exact else (y, basis)
+
+
+class DensePacked:
+    """Dense NVFP4 weights of E expert linears: codes [E, M, K/2] (two E2M1
+    codes per byte, even K low), scales [E, M, K/16] UE4M3, gamma [E]."""
+
+    def __init__(self, codes, scales, gamma):
+        self.codes, self.scales, self.gamma = codes, scales, gamma
+
+
+def pack_dense_nvfp4(w_bf16: np.ndarray) -> DensePacked:
+    """The dense W4A4 control (no pruning, one scale per 16 K), per expert."""
+    w = np.ascontiguousarray(w_bf16, dtype=np.uint16)
+    E, M, K = w.shape
+    codes = np.zeros((E, M, K // 2), np.uint8)
+    scales = np.zeros((E, M, K // 16), np.uint8)
+    gamma = np.zeros(E, np.float32)
+    g1 = np.zeros(1, np.float32)
+    for e in range(E):
+        c = np.zeros((M, K // 2), np.uint8)
+        sc = np.zeros((M, K // 16), np.uint8)
+        lib().oracle_pack_dense_nvfp4(np.ascontiguousarray(w[e]), M, K, c, sc, g1)
+        codes[e], scales[e], gamma[e] = c, sc, g1[0]
+    return DensePacked(codes, scales, gamma)
+
+
+def dense_grouped_gemm(dp: DensePacked, a_codes, a_scales, offsets, gamma_a, want_exact=False):
+    """grouped_gemm for the dense control weights (same activations)."""
+    E, M, K2 = dp.codes.shape
+    K = K2 * 2
+    R = a_codes.shape[0]
+    y = np.zeros((R, M), np.uint16)
+    basis = np.zeros((R, M), np.float64)
+    exact = np.zeros((R, M), np.float64) if want_exact else None
+    lib().oracle_dense_grouped_gemm(np.ascontiguousarray(dp.codes), np.ascontiguousarray(dp.scales),
+                                    np.ascontiguousarray(dp.gamma, np.float32), E, M, K,
+                                    np.ascontiguousarray(a_codes), np.ascontiguousarray(a_scales),
+                                    np.ascontiguousarray(offsets, np.int32),
+                                    np.ascontiguousarray(gamma_a, np.float32), y,
+                                    exact.ctypes.data if want_exact else None, basis.ctypes.data)
     return (y, basis, exact) if want_exact else (y, basis)
 
 

@@ -399,3 +399,84 @@ void oracle_combine(const uint16_t *y_dn, int H, const float *topk_w,
             out[(size_t)t * H + h] = double_to_bf16(s);
         }
 }
+
+/* ------------------------------------------- dense NVFP4 control (no pruning)
+ * The dense W4A4 NVFP4 baseline the paper measures the sparse kernel against
+ * (App. D.2; the "Dense" rows of Tables 10 and 11): every weight kept, one
+ * UE4M3 scale per 16 consecutive K elements (the NVFP4 group), gamma from
+ * Eq. 5 over the whole expert linear, values by Eq. 3.  codes [M][K/2] (low
+ * nibble = even k), scales16 [M][K/16]. */
+void oracle_pack_dense_nvfp4(const uint16_t *w_bf16, int M, int K, uint8_t *codes, uint8_t *scales16,
+                             float *gamma_out) {
+    float amax_t = 0.0f;
+    for (size_t i = 0; i < (size_t)M * K; ++i) {
+        float a = fabsf(bf16_to_float(w_bf16[i]));
+        if (a > amax_t) amax_t = a;
+    }
+    const float gamma = oracle_global_scale(amax_t);
+    *gamma_out = gamma;
+    for (int r = 0; r < M; ++r) {
+        const uint16_t *wr = w_bf16 + (size_t)r * K;
+        for (int b = 0; b < K / 16; ++b) {
+            float amax_b = 0.0f;
+            for (int i = 0; i < 16; ++i) {
+                float a = fabsf(bf16_to_float(wr[16 * b + i]));
+                if (a > amax_b) amax_b = a;
+            }
+            int sc = block_scale_code(gamma, amax_b);
+            scales16[(size_t)r * (K / 16) + b] = (uint8_t)sc;
+            for (int i = 0; i < 8; ++i) {
+                int c0 = quantize_value(bf16_to_float(wr[16 * b + 2 * i]), sc, gamma);
+                int c1 = quantize_value(bf16_to_float(wr[16 * b + 2 * i + 1]), sc, gamma);
+                codes[(size_t)r * (K / 2) + 8 * b + i] = (uint8_t)(c0 | (c1 << 4));
+            }
+        }
+    }
+}
+
+/* Grouped GEMM of the dense control: as oracle_grouped_gemm, with the dense
+ * weight codes and their per-16 scales; the activations are the same NVFP4
+ * rows (per-32 scales), y rounded once to bf16 after alpha_e. */
+void oracle_dense_grouped_gemm(const uint8_t *codes, const uint8_t *scales16, const float *gamma_w, int E,
+                               int M, int K, const uint8_t *a_codes, const uint8_t *a_scales,
+                               const int32_t *offsets, const float *gamma_a, uint16_t *y_bf16,
+                               double *y_exact, double *abs_sum) {
+    double *wq = (double *)malloc(sizeof(double) * (size_t)M * K);
+    double *aq = (double *)malloc(sizeof(double) * (size_t)K);
+    for (int e = 0; e < E; ++e) {
+        int r0 = offsets[e], r1 = offsets[e + 1];
+        if (r1 <= r0) continue;
+        const uint8_t *ce = codes + (size_t)e * M * (K / 2);
+        const uint8_t *se = scales16 + (size_t)e * M * (K / 16);
+        for (int m = 0; m < M; ++m)
+            for (int k = 0; k < K; ++k) {
+                int byte = ce[(size_t)m * (K / 2) + k / 2];
+                int c = (k & 1) ? (byte >> 4) : (byte & 15);
+                wq[(size_t)m * K + k] = oracle_e2m1_value(c) * oracle_ue4m3_value(se[(size_t)m * (K / 16) + k / 16]);
+            }
+        volatile float prod = gamma_w[e] * gamma_a[e];
+        float alpha = 1.0f / prod;
+        for (int r = r0; r < r1; ++r) {
+            for (int k = 0; k < K; ++k) {
+                int byte = a_codes[(size_t)r * (K / 2) + k / 2];
+                int c = (k & 1) ? (byte >> 4) : (byte & 15);
+                aq[k] = oracle_e2m1_value(c) * oracle_ue4m3_value(a_scales[(size_t)r * (K / 32) + k / 32]);
+            }
+            for (int m = 0; m < M; ++m) {
+                const double *wr = wq + (size_t)m * K;
+                double s = 0.0, sa = 0.0;
+                for (int k = 0; k < K; ++k) {
+                    double p = aq[k] * wr[k];
+                    s += p;
+                    sa += fabs(p);
+                }
+                double y = (double)alpha * s;
+                y_bf16[(size_t)r * M + m] = double_to_bf16(y);
+                if (y_exact) y_exact[(size_t)r * M + m] = y;
+                if (abs_sum) abs_sum[(size_t)r * M + m] = fabs((double)alpha) * sa;
+            }
+        }
+    }
+    free(aq);
+    free(wq);
+}
