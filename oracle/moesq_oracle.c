@@ -83,13 +83,37 @@ static float bf16_to_float(uint16_t b) {
     return f;
 }
 
-/* Round to nearest even on the bit pattern; inputs are finite. */
+/* binary64 -> bf16 (1 sign, 8 exponent, 7 fraction bits, the exponent range
+ * of binary32), rounded once to the nearest bf16 number, an exact tie to the
+ * even fraction (the epilogue's FP32 -> BF16 rounding, paper Sec. 3.4 /
+ * App. D.1, applied to the exact sum).  Written from the format's
+ * definition: the spacing of bf16 numbers near |v| is 2^(e-7) for
+ * 2^e <= |v| < 2^(e+1), e >= -126, and 2^-133 below 2^-126 (subnormals);
+ * |v| is divided by that spacing (exact: a power of two), the quotient is
+ * rounded to the nearest integer, ties to even, and scaled back.  Magnitudes
+ * at or above the midpoint between the largest finite bf16 (2 - 2^-7) 2^127
+ * and 2^128 round to infinity (that tie goes to the even neighbour, which is
+ * infinity).  No intermediate binary32 value is formed, so there is no
+ * double rounding.  NaN gives the quiet NaN 0x7FC0. */
 static uint16_t double_to_bf16(double v) {
-    float f = (float)v;
+    if (v != v) return 0x7FC0u;
+    uint16_t sign = signbit(v) ? 0x8000u : 0u;
+    double a = fabs(v);
+    if (a == 0.0) return sign;
+    if (a >= ldexp(2.0 - ldexp(1.0, -8), 127)) return (uint16_t)(sign | 0x7F80u);
+    int e;
+    frexp(a, &e);                        /* a = f * 2^e, 0.5 <= f < 1: 2^(e-1) <= a < 2^e */
+    int lead = e - 1;                    /* exponent of the leading bit */
+    int sp = (lead < -126) ? -133 : lead - 7;
+    double q = ldexp(a, -sp);            /* exact */
+    double n = floor(q);
+    double frac = q - n;                 /* exact: q has at most 53 significant bits */
+    if (frac > 0.5 || (frac == 0.5 && fmod(n, 2.0) != 0.0)) n += 1.0;
+    double r = ldexp(n, sp);             /* a bf16 number, hence exact in binary32 */
+    float f = (float)r;
     uint32_t u;
     memcpy(&u, &f, 4);
-    u += 0x7FFFu + ((u >> 16) & 1u);
-    return (uint16_t)(u >> 16);
+    return (uint16_t)(sign | ((u >> 16) & 0x7FFFu));
 }
 
 uint16_t oracle_bf16_round(double v) { return double_to_bf16(v); }
