@@ -65,7 +65,13 @@ __device__ __forceinline__ void topk_one_token(const float* __restrict__ lr, int
     const uint32_t best = __reduce_max_sync(0xffffffffu, bo);
     const int win = __reduce_min_sync(0xffffffffu, (bo == best && be < E) ? be : 0x7fffffff);
     if (win >= E) {                      // only NaN logits leave no candidate
-      if (lane == 0) record_error(kWhereRoute, kErrFault);
+      // picks j .. k-1 get the sentinel id -1 (weight 0): the counting and
+      // scatter kernels skip it, and the quantiser, SwiGLU and combine
+      // report the slot through the error word
+      if (lane == 0) {
+        record_error(kWhereRoute, kErrFault);
+        for (int jj = j; jj < k; ++jj) { ids_out[jj] = -1; w_out[jj] = 0.0f; }
+      }
       return;
     }
     if ((win & 31) == lane) {
@@ -190,13 +196,17 @@ __global__ void __launch_bounds__(256) route_scatter_kernel(int T, int E, int k,
   for (int i = threadIdx.x; i < nslots; i += blockDim.x) {
     const int tl = i / k;
     const int e = topk_ids[(size_t)t0 * k + i];
-    atomicOr(&bitmap[e * kRouteWords + (tl >> 5)], 1u << (tl & 31));
+    if (e >= 0 && e < E) atomicOr(&bitmap[e * kRouteWords + (tl >> 5)], 1u << (tl & 31));
   }
   __syncthreads();
   for (int i = threadIdx.x; i < nslots; i += blockDim.x) {
     const int tl = i / k;
     const int slot = t0 * k + i;
     const int e = topk_ids[slot];
+    if (e < 0 || e >= E) {               // not counted: the slot has no row
+      slot_to_row[slot] = -1;
+      continue;
+    }
     int rank = 0;
 #pragma unroll
     for (int w = 0; w < kRouteWords; ++w) {
@@ -273,7 +283,10 @@ __global__ void __launch_bounds__(1024) route_finish_kernel(int T, int E, int k,
   for (int i = threadIdx.x; i < nslots; i += blockDim.x) {
     const int tl = i / k;
     const int e = topk_ids[i];
-    if (e < 0 || e >= E) continue;
+    if (e < 0 || e >= E) {               // not counted: the slot has no row
+      slot_to_row[i] = -1;
+      continue;
+    }
     int rank = 0;
     for (int w = 0; w < (tl >> 5); ++w) rank += __popc(bitmap[e * words + w]);
     rank += __popc(bitmap[e * words + (tl >> 5)] & ((1u << (tl & 31)) - 1u));

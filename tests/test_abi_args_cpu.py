@@ -85,6 +85,13 @@ def test_routing_checks(L):
     need = L.moesq_route_workspace_bytes(8, 4)
     assert L.moesq_route_permute(ptr(), ctypes.byref(rt), ptr(), max(0, need - 1), None) == WORKSPACE
     assert L.moesq_route_permute(ptr(), ctypes.byref(rt), None, need, None) == WORKSPACE
+    assert L.moesq_route_permute(ptr(), ctypes.byref(routing(T=0)), ptr(), 1 << 20, None) == SHAPE
+    assert L.moesq_route_permute(ptr(), ctypes.byref(routing(E=513, k=8)), ptr(), 1 << 30, None) == SHAPE
+    assert L.moesq_route_permute(ptr(), ctypes.byref(routing(E=64, k=33)), ptr(), 1 << 30, None) == SHAPE
+    # the allocation-free variant: the same checks, and tokens beyond its static scratch
+    assert L.moesq_route_permute_noalloc(ptr(), ctypes.byref(routing(k=0)), None) == SHAPE
+    assert L.moesq_route_permute_noalloc(None, ctypes.byref(rt), None) == INVALID
+    assert L.moesq_route_permute_noalloc(ptr(), ctypes.byref(routing(T=16385, E=8, k=2)), None) == SHAPE
 
 
 def test_quantise_swiglu_combine_checks(L):
