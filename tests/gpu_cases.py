@@ -89,3 +89,78 @@ def gemm_tolerance_ok(y_gpu_bits, y_ref_bits, basis):
     bound = 1e-3 * basis + L.bf16_ulp(r) + 1e-30
     bad = err > bound
     return (not bad.any()), err, bound, bad
+
+
+def expert_weights_host(seed, linear, e, M, K):
+    """One expert's bf16 weight bits on the host, drawn by the seeded
+    generator's torch path on the GPU (same bits as the numpy path, which
+    takes seconds per Kimi-sized expert on the host)."""
+    torch = torch_mod()
+    w = S.expert_weights_bf16_torch(seed, linear, int(e), M, K, "cuda")
+    return w.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def oracle_pack_experts(seed, linear, E, M, K, experts):
+    """Oracle storage form of an E-expert stack in which only `experts` hold
+    their seeded weights (the other experts' tensors stay zero and unread):
+    the oracle side of a token sample at full size."""
+    import oracle as O
+    experts = [int(e) for e in experts]
+    pk = O.pack_weights(np.stack([expert_weights_host(seed, linear, e, M, K) for e in experts]))
+    full = O.Packed(np.zeros((E, M, K // 4), np.uint8), np.zeros((E, M, K // 16), np.uint8),
+                    np.zeros((E, M, K // 32), np.uint8), np.ones(E, np.float32))
+    full.values[experts], full.mask[experts], full.scales[experts], full.gamma[experts] = \
+        pk.values, pk.mask, pk.scales, pk.gamma
+    return full
+
+
+# ---------------------------------------------------------------- requantisation check with a decision band
+E2M1_DECISION_POINTS = (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0)   # midpoints of the App. A, Fig. 3 grid
+
+# Relative band around a decision point inside which a binary32 SiLU with
+# the hardware exponential and divide (a few tens of ulp for |g| <= 16, below
+# 2^-18 relative) may put h on the other side of the oracle's binary64 h;
+# 2^-16 leaves a factor of 4 over that.
+SWIGLU_BAND = 2.0 ** -16
+
+
+def _ue4m3_decisions():
+    """Midpoints between consecutive UE4M3 values (codes 0..126): the points
+    where Eq. 5's scale code changes."""
+    import oracle as O
+    v = np.array([O.ue4m3_value(c) for c in range(127)], np.float64)
+    return (v[:-1] + v[1:]) / 2
+
+
+def _near(x, points, band):
+    """|x - p| <= band * p for the decision point p nearest x (x >= 0)."""
+    pts = np.asarray(points, np.float64)
+    i = np.clip(np.searchsorted(pts, x), 1, pts.size - 1)
+    d = np.minimum(np.abs(x - pts[i - 1]) / pts[i - 1], np.abs(x - pts[i]) / pts[i])
+    return d <= band
+
+
+def requant_mismatches(h, gamma_rows, os_, oc, gs, gc, band=SWIGLU_BAND):
+    """Compares a requantisation (gs scale codes [R, I/32], gc code bytes
+    [R, I/2]) with the oracle's (os_, oc) of h (binary32 [R, I]) under the
+    per-row global scales gamma_rows [R].  A scale code may differ only where
+    gamma * amax_b / 6 lies within `band` of a UE4M3 decision point (a
+    changed scale then frees its whole block); under an equal scale a value
+    code may differ only where |h| / s_b lies within `band` of an E2M1
+    decision point.  Returns (bad_scale [R, I/32], bad_code [R, I/32, 32],
+    scale_diff, code_diff)."""
+    import oracle as O
+    R, I = h.shape
+    hb = h.astype(np.float64).reshape(R, I // 32, 32)
+    g = np.asarray(gamma_rows, np.float32)
+    x_s = g.astype(np.float64)[:, None] * np.abs(hb).max(-1) / 6.0
+    scale_diff = gs != os_
+    bad_scale = scale_diff & ~_near(x_s, _ue4m3_decisions(), band)
+    sv = np.vectorize(O.ue4m3_value)(os_).astype(np.float32)
+    s_b = (sv / g[:, None]).astype(np.float64)
+    q = np.abs(hb) / np.where(s_b > 0, s_b, np.inf)[..., None]
+    code_free = _near(q, E2M1_DECISION_POINTS, band)
+    nib = lambda c: np.stack([c & 15, c >> 4], -1).reshape(R, I // 32, 32)   # noqa: E731
+    code_diff = nib(gc) != nib(oc)
+    bad_code = code_diff & ~code_free & ~scale_diff[..., None]
+    return bad_scale, bad_code, scale_diff, code_diff

@@ -6,8 +6,8 @@ import pytest
 import layouts as L
 import oracle as O
 import synthetic as S
-from gpu_cases import (act_rows_from_compact, gemm_tolerance_ok, pack_gpu_from_np, pack_gpu_generated,
-                       packed_from_oracle, to_dev, to_np, weights_np)
+from gpu_cases import (act_rows_from_compact, expert_weights_host, gemm_tolerance_ok, pack_gpu_from_np,
+                       pack_gpu_generated, packed_from_oracle, to_dev, to_np, weights_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -117,16 +117,25 @@ def test_gemm_full_path_30b_class(cuda_lib):
         assert ok, (e, err.max())
 
 
-@pytest.mark.parametrize("T", [1, 64])
-def test_gemm_kimi_decode_full_size_sampled(cuda_lib, T):
-    """Kimi-shaped gate_up at full size (E=384, K=7168, M=4096): every output
-    of 2 sampled experts against the oracle."""
+@pytest.fixture(scope="module")
+def kimi_gate_up(cuda_lib):
+    """Kimi-shaped gate_up weights (E=384, M=4096, K=7168), drawn and packed on
+    the GPU once for the decode tests of this module."""
+    return pack_gpu_generated(cuda_lib, 21, 0, 384, 4096, 7168, chunk=4)
+
+
+@pytest.mark.parametrize("T", [1, 16, 64, 256])
+def test_gemm_kimi_decode_full_size_sampled(cuda_lib, kimi_gate_up, T):
+    """Kimi-shaped gate_up at full size (E=384, K=7168, M=4096), the decode
+    token counts: CUDA route, dispatch-quantise and GEMM; every output of four
+    sampled experts (the heaviest, the lightest and two others) against the
+    oracle, and their packed values bit for bit."""
     torch = pytest.importorskip("torch")
     m = cuda_lib
     E, M, K, k = 384, 4096, 7168, 8
-    pw = pack_gpu_generated(m, 21, 0, E, M, K, chunk=4)
-    x = S.activations_bf16_np(21, T, K)
-    lg = S.uniform_logits_np(21, T, E)
+    pw = kimi_gate_up
+    x = S.activations_bf16_np(21 + T, T, K)
+    lg = S.uniform_logits_np(21 + T, T, E)
     rt = O.route(lg, k)
     ga = np.full(E, O.act_global_scale(x), np.float32)
     rb = m.RoutingBuffers(T, E, k)
@@ -139,16 +148,19 @@ def test_gemm_kimi_decode_full_size_sampled(cuda_lib, T):
     yg_all = to_np(y)
     ro = L.aligned_rows(rt.counts)
     used = np.nonzero(rt.counts)[0]
-    for e in (used[0], used[-1]):
+    rng = np.random.default_rng(T)
+    pick = {int(used[np.argmax(rt.counts[used])]), int(used[np.argmin(rt.counts[used])])}
+    pick.update(int(e) for e in rng.choice(used, size=min(2, used.size), replace=False))
+    for e in sorted(pick):
         n = int(rt.counts[e])
-        pk = O.pack_weights(S.expert_weights_bf16_np(21, 0, int(e), M, K)[None])
+        pk = O.pack_weights(expert_weights_host(21, 0, e, M, K)[None])
         assert (to_np(pw.values[e]) == pk.values[0]).all()
         s0 = rt.offsets[e]
         toks = rt.sorted_to_slot[s0:s0 + n] // k
         c, s = O.quantize_rows_bf16(x[toks], ga[e])
         y_ref, basis = O.grouped_gemm(pk, c, s, np.array([0, n], np.int32), ga[e:e + 1])
         ok, err, bound, bad = gemm_tolerance_ok(yg_all[ro[e]:ro[e] + n], y_ref, basis)
-        assert ok, (e, err.max())
+        assert ok, (T, e, n, err.max())
 
 
 def test_gemm_rejects_inconsistent_counts(cuda_lib):
@@ -274,7 +286,7 @@ def test_gemm_kimi_prefill_down_full_size_sampled(cuda_lib):
     for e in (heavy, light):
         n = int(rt.counts[e])
         idx = _prefill_rows(n) if e == heavy else np.arange(n)
-        pk = O.pack_weights(S.expert_weights_bf16_np(31, 1, e, M, K)[None])
+        pk = O.pack_weights(expert_weights_host(31, 1, e, M, K)[None])
         s0 = rt.offsets[e]
         toks = rt.sorted_to_slot[s0:s0 + n][idx] // k
         c, s = O.quantize_rows_bf16(x[toks], ga[e])

@@ -7,7 +7,7 @@ import pytest
 import layouts as L
 import oracle as O
 import synthetic as S
-from gpu_cases import (pack_gpu_from_np, pack_gpu_generated, to_dev, to_np, weights_np)
+from gpu_cases import (pack_gpu_from_np, pack_gpu_generated, requant_mismatches, to_dev, to_np, weights_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -120,17 +120,24 @@ def test_quantize_dispatch_bit_exact(cuda_lib, T, E, k, K):
     assert (L.mma_to_scales(to_np(scales), rb.rows_cap, K)[rows] == os_).all()
 
 
-def test_swiglu_quant_matches_oracle(cuda_lib):
+@pytest.mark.parametrize("I,sigma", [(512, 2.0), (2048, 6.0)])
+def test_swiglu_quant_matches_oracle(cuda_lib, I, sigma):
+    """SwiGLU + requantisation against the oracle, complete: every scale code
+    equal unless the block's gamma * amax / 6 lies within SWIGLU_BAND of a
+    UE4M3 decision point; under an equal scale code every E2M1 code equal
+    unless h / s_b lies within SWIGLU_BAND of an E2M1 decision point; no
+    other difference is allowed (gpu_cases.requant_mismatches)."""
     m = cuda_lib
-    T, E, k, I = 48, 8, 2, 512
+    T, E, k = 48, 8, 2
     lg = S.uniform_logits_np(9, T, E)
     rt = O.route(lg, k)
     R = T * k
-    rng = np.random.default_rng(9)
-    y_c = S.f32_to_bf16_bits_np(rng.normal(0, 2, size=(R, 2 * I)).astype(np.float32))
-    gh = np.full(E, O.global_scale(np.abs(O.swiglu(y_c)).max()), np.float32)
-    gh[3] *= np.float32(0.5)
+    rng = np.random.default_rng(9 + I)
+    y_c = S.f32_to_bf16_bits_np(rng.normal(0, sigma, size=(R, 2 * I)).astype(np.float32))
     h = O.swiglu(y_c)
+    gh = np.full(E, O.global_scale(np.abs(h).max()), np.float32)
+    gh[3] *= np.float32(0.5)
+    gh[5] *= np.float32(3.0)
     oc, os_ = O.requantize_rows(h, rt, gh)
     rb = m.RoutingBuffers(T, E, k)
     m.moesq_route_permute(to_dev(lg), rb)
@@ -139,12 +146,15 @@ def test_swiglu_quant_matches_oracle(cuda_lib):
     y_rows[rows] = y_c
     hc, hs = m.act_buffers(rb.rows_cap, I)
     m.moesq_swiglu_quant(to_dev(y_rows), I, rb, to_dev(gh), hc, hs)
+    assert m.moesq_get_device_error()[0] == 0
     gc = to_np(hc)[rows]
     gs = L.mma_to_scales(to_np(hs), rb.rows_cap, I)[rows]
-    # binary32 SiLU on the GPU vs binary64 in the oracle: a code may flip at
-    # an exact rounding boundary; scales and almost all codes agree
-    assert (gs == os_).mean() > 0.999
-    assert (gc == oc).mean() > 0.999
+
+    bad_scale, bad_code, scale_diff, code_diff = requant_mismatches(h, gh[rt.expert_of_sorted()], os_, oc, gs, gc)
+    assert not bad_scale.any(), np.argwhere(bad_scale)[:5]
+    assert not bad_code.any(), (np.argwhere(bad_code)[:5], int(bad_code.sum()))
+    # the allowance is rare: the band covers a tiny part of the value range
+    assert scale_diff.mean() < 1e-2 and code_diff.mean() < 1e-3
 
 
 # ---------------------------------------------------------------- quantiser near the E2M1 decision points

@@ -24,7 +24,10 @@ def _route_both(m, lg, T, E, k):
     return ref, new
 
 
-@pytest.mark.parametrize("T,E,k", [(300, 128, 8), (4096, 384, 8)])
+# Both cases take the multi-kernel routing path (T > 512 tokens), the one
+# that keeps per-block expert counts in the static scratch; the second fills
+# the scratch to its limit (16384 tokens = 128 blocks, 512 experts).
+@pytest.mark.parametrize("T,E,k", [(4096, 384, 8), (16384, 512, 8)])
 def test_noalloc_routing_equals_workspace_routing_twice(cuda_lib, T, E, k):
     m = cuda_lib
     # two calls in a row with different logits: the second must not see the
