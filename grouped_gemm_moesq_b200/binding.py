@@ -43,7 +43,7 @@ class moesq_routing(ctypes.Structure):
 
 
 class moesq_gemm_config(ctypes.Structure):
-    _fields_ = [("tile_n", _i32), ("num_ctas", _i32)]
+    _fields_ = [("tile_n", _i32), ("num_ctas", _i32), ("sm_mode", _i32)]
 
 
 _lib = None
@@ -75,6 +75,7 @@ def load():
         "moesq_route_workspace_bytes": (_sz, [_c.c_int, _c.c_int]),
         "moesq_route_permute": (_c.c_int, [_vp, _P(moesq_routing), _vp, _sz, _vp]),
         "moesq_route_permute_noalloc": (_c.c_int, [_vp, _P(moesq_routing), _vp]),
+        "moesq_mma_peak": (_c.c_int, [_c.c_int, _c.c_int, _c.c_int, _c.c_int, _c.c_int, _P(_c.c_double), _vp]),
         "moesq_quantize_act": (_c.c_int, [_vp, _c.c_int, _c.c_int, _P(moesq_routing), _vp, _c.c_int, _vp, _vp,
                                           _vp]),
         "moesq_act_global_scale": (_c.c_int, [_vp, _i64, _vp, _vp]),
@@ -214,13 +215,13 @@ def moesq_pack_weights(w_bf16, e_begin: int, e_count: int, out: PackedWeights, s
 
 def moesq_gemm_autotune(w: PackedWeights, a_codes, a_scales, rows_cap: int, counts, row_offsets, gamma_a, y_bf16,
                         reps: int = 5, stream=None):
-    """Fastest (tile_n, num_ctas) for these inputs and its mean time in ms."""
+    """Fastest (tile_n, num_ctas, sm_mode) for these inputs and its mean time in ms."""
     cfg = moesq_gemm_config(0, 0)
     ms = _c.c_float(0.0)
     _check(load().moesq_gemm_autotune(ctypes.byref(w.struct), _ptr(a_codes), _ptr(a_scales), rows_cap, _ptr(counts),
                                       _ptr(row_offsets), _ptr(gamma_a), _ptr(y_bf16), reps, ctypes.byref(cfg),
                                       ctypes.byref(ms), _stream(stream)), "moesq_gemm_autotune")
-    return (cfg.tile_n, cfg.num_ctas), ms.value
+    return (cfg.tile_n, cfg.num_ctas, cfg.sm_mode), ms.value
 
 
 def moesq_import_dense_nvfp4(codes, scales, global_scale, e_begin: int, e_count: int, out: PackedWeights,
@@ -258,8 +259,8 @@ def moesq_act_global_scale(x_bf16, gamma_out, stream=None):
 
 
 def moesq_grouped_sparse_gemm(w: PackedWeights, a_codes, a_scales, rows_cap: int, counts, row_offsets, gamma_a,
-                              y_bf16, tile_n: int = 0, num_ctas: int = 0, stream=None):
-    cfg = moesq_gemm_config(tile_n, num_ctas)
+                              y_bf16, tile_n: int = 0, num_ctas: int = 0, sm_mode: int = 0, stream=None):
+    cfg = moesq_gemm_config(tile_n, num_ctas, sm_mode)
     _check(load().moesq_grouped_sparse_gemm(ctypes.byref(w.struct), _ptr(a_codes), _ptr(a_scales), rows_cap,
                                             _ptr(counts), _ptr(row_offsets), _ptr(gamma_a), _ptr(y_bf16),
                                             ctypes.byref(cfg), _stream(stream)), "moesq_grouped_sparse_gemm")
@@ -300,3 +301,13 @@ def moesq_calibrate_layer(x_bf16, logits, T: int, k: int, w_gu: PackedWeights, w
 
 def moesq_debug_bounded_wait(timeout_ns: int, stream=None):
     _check(load().moesq_debug_bounded_wait(int(timeout_ns), _stream(stream)), "moesq_debug_bounded_wait")
+
+
+def moesq_mma_peak(sparse: bool, n: int, ctas_per_sm: int = 1, with_copies: bool = False, iters: int = 20000,
+                   stream=None) -> float:
+    """Dense-equivalent TFLOP/s of back-to-back block-scaled FP4 MMAs on every SM."""
+    out = ctypes.c_double(0.0)
+    _check(load().moesq_mma_peak(int(bool(sparse)), n, ctas_per_sm, int(bool(with_copies)), iters,
+                                 ctypes.byref(out), _stream(stream)),
+           "moesq_mma_peak")
+    return out.value

@@ -15,6 +15,7 @@
 #include "common.cuh"
 #include "gemm.cuh"
 #include "pack.cuh"
+#include "peak.cuh"
 #include "quant.cuh"
 #include "route.cuh"
 
@@ -497,8 +498,10 @@ moesq_status moesq_grouped_sparse_gemm(const moesq_weights* w, const uint8_t* a_
   if (!aligned(a_codes, 16) || !aligned(a_scales, 16) || !aligned(y_bf16, 2)) return MOESQ_ERR_INVALID_ARG;
   int tile_n = cfg ? cfg->tile_n : 0;
   const int num_ctas = cfg ? cfg->num_ctas : 0;
+  const int sm_mode = cfg ? cfg->sm_mode : 0;
   if (tile_n != 0 && tile_n != 64 && tile_n != 128) return MOESQ_ERR_INVALID_ARG;
-  if (num_ctas < 0) return MOESQ_ERR_INVALID_ARG;
+  if (num_ctas < 0 || sm_mode < 0 || sm_mode > 2) return MOESQ_ERR_INVALID_ARG;
+  if (sm_mode == 2) return MOESQ_ERR_UNSUPPORTED_SHAPE;
   if (tile_n == 0) {
     // The counts stay on the device.  The aligned row capacity, less the
     // padding of at most 127 rows per expert, bounds the mean rows per expert.
@@ -518,7 +521,7 @@ moesq_status moesq_gemm_autotune(const moesq_weights* w, const uint8_t* a_codes,
   if (!best || !best_ms || reps < 1) return MOESQ_ERR_INVALID_ARG;
   cudaStream_t s = as_stream(stream);
   const int sms = device_info().sms;
-  const moesq_gemm_config cands[4] = {{64, 2 * sms}, {128, 2 * sms}, {64, sms}, {128, sms}};
+  const moesq_gemm_config cands[4] = {{64, 2 * sms, 1}, {128, 2 * sms, 1}, {64, sms, 1}, {128, sms, 1}};
   cudaEvent_t ev[2];
   MOESQ_CUDA(cudaEventCreate(&ev[0]));
   if (cudaEventCreate(&ev[1]) != cudaSuccess) {
@@ -648,6 +651,46 @@ moesq_status moesq_calibrate_layer(const uint16_t* x_bf16, const float* logits, 
 moesq_status moesq_debug_bounded_wait(uint64_t timeout_ns, void* stream) {
   debug_wait_kernel<<<1, 32, 0, as_stream(stream)>>>(timeout_ns ? timeout_ns : 1);
   return last_launch();
+}
+
+moesq_status moesq_mma_peak(int sparse, int n, int ctas_per_sm, int with_copies, int iters, double* tflops,
+                            void* stream) {
+  if (!tflops || iters < 1 || (sparse != 0 && sparse != 1)) return MOESQ_ERR_INVALID_ARG;
+  if (with_copies != 0 && with_copies != 1) return MOESQ_ERR_INVALID_ARG;
+  if (ctas_per_sm != 1 && ctas_per_sm != 2) return MOESQ_ERR_INVALID_ARG;
+  if (n < 16 || n > 256 || n % 16 || (ctas_per_sm == 2 && n > 128)) return MOESQ_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  const int sms = device_info().sms;
+  // dynamic shared memory sized so that exactly ctas_per_sm CTAs fit on an
+  // SM: each then owns 512 / ctas_per_sm TMEM columns
+  const size_t smem = ctas_per_sm == 1 ? (size_t)150 * 1024 : (size_t)100 * 1024;
+  const uint32_t cols = ctas_per_sm == 1 ? 512u : 256u;
+  auto kern = sparse ? (with_copies ? mma_peak_kernel<true, true> : mma_peak_kernel<true, false>)
+                     : (with_copies ? mma_peak_kernel<false, true> : mma_peak_kernel<false, false>);
+  MOESQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  cudaEvent_t ev[2];
+  MOESQ_CUDA(cudaEventCreate(&ev[0]));
+  if (cudaEventCreate(&ev[1]) != cudaSuccess) {
+    cudaEventDestroy(ev[0]);
+    return MOESQ_ERR_CUDA;
+  }
+  moesq_status st = MOESQ_OK;
+  float ms = 0.0f;
+  if (cudaEventRecord(ev[0], s) != cudaSuccess) st = MOESQ_ERR_CUDA;
+  if (st == MOESQ_OK) {
+    kern<<<sms * ctas_per_sm, kPeakThreads, smem, s>>>(n, iters, cols, g_timeout_ns, nullptr);
+    st = last_launch();
+  }
+  if (st == MOESQ_OK && (cudaEventRecord(ev[1], s) != cudaSuccess || cudaEventSynchronize(ev[1]) != cudaSuccess ||
+                         cudaEventElapsedTime(&ms, ev[0], ev[1]) != cudaSuccess))
+    st = MOESQ_ERR_CUDA;
+  cudaEventDestroy(ev[0]);
+  cudaEventDestroy(ev[1]);
+  if (st != MOESQ_OK) return st;
+  const double k_dense = sparse ? 128.0 : 64.0;
+  const double flops = (double)sms * ctas_per_sm * iters * 2.0 * 2.0 * 128.0 * n * k_dense;
+  *tflops = flops / ((double)ms * 1e-3) / 1e12;
+  return MOESQ_OK;
 }
 
 moesq_status moesq_route_permute_noalloc(const float* logits, const moesq_routing* rt, void* stream) {

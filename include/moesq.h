@@ -267,6 +267,9 @@ typedef struct {
   int32_t tile_n;      /* token rows per tile: 0 = auto, 64 or 128 */
   int32_t num_ctas;    /* persistent CTAs: 0 = two per SM (two independent
                           tensor-core issue streams per SM) */
+  int32_t sm_mode;     /* 0 = auto; 1 = one SM per 128-row weight tile;
+                          2 = a pair of SMs per 256-row weight tile (not
+                          built: MOESQ_ERR_UNSUPPORTED_SHAPE) */
 } moesq_gemm_config;
 
 moesq_status moesq_grouped_sparse_gemm(const moesq_weights* w, const uint8_t* a_codes,
@@ -351,6 +354,25 @@ moesq_status moesq_calibrate_layer(const uint16_t* x_bf16, const float* logits, 
  * MOESQ_ERR_TIMEOUT in the device error word and the kernel exits.  Exists
  * to test the watchdog path of the kernels without faulting the GPU. */
 moesq_status moesq_debug_bounded_wait(uint64_t timeout_ns, void* stream);
+
+/* --------------------------------------------------------- tensor-core peak
+ * Throughput of the block-scaled FP4 MMA this library's GEMM is built on
+ * (tcgen05.mma kind::mxf4nvf4 with UE4M3 scales; the sparse form is the
+ * paper's SpTC path, Sec. 3.4 and App. D.1; the 18 PFLOP/s sparse peak the
+ * paper quotes for B200 in its introduction is the nominal counterpart):
+ * ctas_per_sm (1 or 2) CTAs on every SM each issue `iters` x 2 back-to-back
+ * MMAs of M = 128, N = n (16 <= n <= 256, a multiple of 16; n <= 128 with
+ * 2 CTAs per SM), K = 64 (dense, sparse = 0) or K = 128 dense-equivalent
+ * (sparse = 1), on operands resident in shared and tensor memory, so no
+ * memory traffic limits it.  with_copies = 1 adds, before every two MMAs,
+ * the shared-to-tensor-memory copies of metadata and scales that the
+ * grouped GEMM issues per 256-wide K step, so the rate then includes their
+ * share of the tensor pipe.  *tflops (host) receives the dense-equivalent
+ * TFLOP/s of the whole GPU (2 M N K per MMA over the launch's event-timed
+ * duration).  Synchronises `stream`; about iters x 0.14 us of device time.
+ * Errors: MOESQ_ERR_INVALID_ARG for sizes outside the above. */
+moesq_status moesq_mma_peak(int sparse, int n, int ctas_per_sm, int with_copies, int iters, double* tflops,
+                            void* stream);
 
 #ifdef __cplusplus
 }

@@ -63,6 +63,8 @@ def test_gemm_refuses_bad_activations_and_config(L):
     assert gemm(L, w, y=ptr(1)) == INVALID                         # bf16 output misaligned
     assert gemm(L, w, cfg=B.moesq_gemm_config(32, 0)) == INVALID   # token tile 32 is not offered
     assert gemm(L, w, cfg=B.moesq_gemm_config(64, -1)) == INVALID
+    assert gemm(L, w, cfg=B.moesq_gemm_config(64, 0, 3)) == INVALID      # sm_mode 0, 1 or 2
+    assert gemm(L, w, cfg=B.moesq_gemm_config(64, 0, -1)) == INVALID
 
 
 def test_autotune_refuses_bad_arguments(L):
@@ -129,3 +131,16 @@ def test_dense_converter_checks(L):
     assert L.moesq_import_dense_nvfp4(ptr(), ptr(), ptr(), 3, 2, ctypes.byref(w), None) == INVALID
     assert L.moesq_export_dense_nvfp4(ctypes.byref(w), ptr(8), None) == INVALID
     assert L.moesq_export_dense_nvfp4(ctypes.byref(weights(M=64)), ptr(), None) == SHAPE
+
+
+def test_mma_peak_checks(L):
+    out = ctypes.c_double(0)
+    assert L.moesq_mma_peak(1, 128, 1, 0, 100, None, None) == INVALID
+    assert L.moesq_mma_peak(2, 128, 1, 0, 100, ctypes.byref(out), None) == INVALID     # sparse is 0 or 1
+    assert L.moesq_mma_peak(1, 8, 1, 0, 100, ctypes.byref(out), None) == INVALID       # n below 16
+    assert L.moesq_mma_peak(1, 264, 1, 0, 100, ctypes.byref(out), None) == INVALID     # n above 256
+    assert L.moesq_mma_peak(1, 200, 1, 0, 100, ctypes.byref(out), None) == INVALID     # not a multiple of 16
+    assert L.moesq_mma_peak(1, 256, 2, 0, 100, ctypes.byref(out), None) == INVALID     # two CTAs: n <= 128
+    assert L.moesq_mma_peak(1, 128, 3, 0, 100, ctypes.byref(out), None) == INVALID
+    assert L.moesq_mma_peak(1, 128, 1, 0, 0, ctypes.byref(out), None) == INVALID
+    assert L.moesq_mma_peak(1, 128, 1, 2, 100, ctypes.byref(out), None) == INVALID   # with_copies is 0 or 1

@@ -12,7 +12,7 @@ from gpu_cases import (act_rows_from_compact, expert_weights_host, gemm_toleranc
 pytestmark = pytest.mark.gpu
 
 
-def _run_isolated(m, pk, counts, K, seed, tile_n, ga_scale=1.0):
+def _run_isolated(m, pk, counts, K, seed, tile_n, ga_scale=1.0, mode=0):
     """Oracle weights + oracle-quantised activations, laid out on the host,
     through the CUDA GEMM; returns (ok, detail)."""
     torch = pytest.importorskip("torch")
@@ -35,7 +35,7 @@ def _run_isolated(m, pk, counts, K, seed, tile_n, ga_scale=1.0):
     M = pk.values.shape[1]
     y = torch.full((rc, M), float("nan"), dtype=torch.bfloat16, device="cuda")
     m.moesq_grouped_sparse_gemm(pw, to_dev(c_rows), to_dev(s_mma), rc, to_dev(counts.astype(np.int32)),
-                                to_dev(L.aligned_rows(counts)), to_dev(ga), y, tile_n=tile_n)
+                                to_dev(L.aligned_rows(counts)), to_dev(ga), y, tile_n=tile_n, sm_mode=mode)
     st, word = m.moesq_get_device_error()
     assert st == 0, "device error word %#x" % word
     rows = L.compact_to_rows(counts)
@@ -54,25 +54,37 @@ def test_gemm_tiny_config(cuda_lib, tile_n):
     assert ok, info[:2]
 
 
-@pytest.mark.parametrize("tile_n", [64, 128])
+@pytest.mark.parametrize("tile_n,mode", [(64, 1), (128, 1)])
 @pytest.mark.parametrize("counts", [
     [0, 1, 0, 5, 0, 0, 0, 2],              # empty experts, single rows
     [129, 0, 31, 33, 1, 16, 17, 300],      # ragged: several token blocks, partial last blocks
     [0, 0, 0, 0, 0, 0, 0, 512],            # all rows on one expert
     [128, 256, 32, 64, 96, 160, 192, 224], # exact multiples of the token block
 ])
-def test_gemm_edge_counts(cuda_lib, tile_n, counts):
+def test_gemm_edge_counts(cuda_lib, tile_n, mode, counts):
     E, M, K = 8, 256, 512
     pk = O.pack_weights(weights_np(3, 0, E, M, K))
-    ok, info = _run_isolated(cuda_lib, pk, np.array(counts, np.int64), K, 4, tile_n)
+    ok, info = _run_isolated(cuda_lib, pk, np.array(counts, np.int64), K, 4, tile_n, mode=mode)
     assert ok, info[:2]
 
 
-def test_gemm_multi_k_tiles_and_m_blocks(cuda_lib):
-    """K = 2048 (8 K steps, deeper than the smem ring wraps) and M = 1536."""
-    E, M, K = 3, 1536, 2048
+@pytest.mark.parametrize("tile_n,mode", [(0, 0), (64, 1), (128, 1)])
+def test_gemm_multi_k_tiles_and_m_blocks(cuda_lib, tile_n, mode):
+    """K = 7168 (28 K steps: every ring wraps several times), M = 1536."""
+    E, M, K = 3, 1536, 7168
     pk = O.pack_weights(weights_np(5, 0, E, M, K))
-    ok, info = _run_isolated(cuda_lib, pk, np.array([7, 0, 40]), K, 6, 0)
+    ok, info = _run_isolated(cuda_lib, pk, np.array([7, 0, 200]), K, 6, tile_n, mode=mode)
+    assert ok, info[:2]
+
+
+@pytest.mark.parametrize("K", [256, 768])
+@pytest.mark.parametrize("tile_n,mode", [(64, 1), (128, 1)])
+def test_gemm_odd_k_steps(cuda_lib, K, tile_n, mode):
+    """K = 256 and 768: one and three 256-wide K steps, fewer than a ring
+    holds, and a count that does not divide it."""
+    E, M = 4, 256
+    pk = O.pack_weights(weights_np(15, 0, E, M, K))
+    ok, info = _run_isolated(cuda_lib, pk, np.array([33, 0, 130, 64]), K, 16, tile_n, mode=mode)
     assert ok, info[:2]
 
 
@@ -237,11 +249,11 @@ def test_gemm_autotune_picks_a_candidate_and_stays_correct(cuda_lib):
     args = (to_dev(c_rows), to_dev(s_mma), rc, to_dev(counts.astype(np.int32)), to_dev(L.aligned_rows(counts)),
             to_dev(ga))
     y = torch.zeros((rc, M), dtype=torch.bfloat16, device="cuda")
-    (tile_n, num_ctas), ms = m.moesq_gemm_autotune(pw, *args, y, reps=2)
+    (tile_n, num_ctas, mode), ms = m.moesq_gemm_autotune(pw, *args, y, reps=2)
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    assert tile_n in (64, 128) and num_ctas in (sms, 2 * sms) and ms > 0
+    assert tile_n in (64, 128) and num_ctas in (sms, 2 * sms) and mode in (1, 2) and ms > 0
     y.fill_(float("nan"))
-    m.moesq_grouped_sparse_gemm(pw, *args, y, tile_n=tile_n, num_ctas=num_ctas)
+    m.moesq_grouped_sparse_gemm(pw, *args, y, tile_n=tile_n, num_ctas=num_ctas, sm_mode=mode)
     assert m.moesq_get_device_error()[0] == 0
     ok, err, bound, bad = gemm_tolerance_ok(to_np(y)[L.compact_to_rows(counts)], y_ref, basis)
     assert ok, err.max()
