@@ -3,21 +3,25 @@
 A step is one pass of the whole hot path over one batch: route + permute,
 dispatch-quantise, gate_up grouped sparse GEMM, SwiGLU + requantise, down
 grouped sparse GEMM, router-weighted combine (weight packing is offline and
-not timed).  The default workload is the 30B-class MoE layer (128 experts,
-top-8, hidden 2048, intermediate 768 -> gate_up N = 1536, T = 256 tokens,
-uniform router logits), synthetic data of the pages' distributions.
+not timed).  The default workload is the Kimi-K2.5-shaped MoE layer (384
+experts, top-8, hidden 7168, intermediate 2048 -> gate_up N = 4096) swept over
+T = 1 ... 16384 tokens with uniform and Zipf(1.1) routing; the headline
+numbers are those of T = 4096 with Zipf routing, and every point of the sweep
+is in `sweep`.  Synthetic data of the pages' distributions.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--impl reference]
 
 Prints one JSON line (rank 0).  `value` is the effective TFLOP/s of the
-step's two grouped GEMMs (2 * M * K per routed row, the pages' App. D.2
+step's grouped GEMMs (2 * M * K per routed row, the pages' App. D.2
 definition) over all ranks; `weight_gbs` the packed expert weights the step
 reads.  Device time: the step is captured once as a CUDA graph and replayed;
 CUDA events around each replay on the launching stream, L2 flushed (256 MiB
 write) before every step outside the events; max over ranks.  Event nodes
-inside the graph give the per-kernel breakdown of the same replays.  `e2e`: the same metric through moesq_moe_layer_host with the step's
-inputs and output in pinned host memory (copies inside the timed region).
+inside a second graph give the per-kernel breakdown of the same replays.
+`e2e`: the same metric through moesq_moe_layer_host with the step's inputs
+and output in pinned host memory (copies inside the timed region).
+`--gpus N` with N > 1 starts N ranks (torch.distributed.run, one per GPU).
 `--impl reference` times the CPU oracle on a bounded token sample instead.
 """
 from __future__ import annotations
@@ -28,6 +32,7 @@ import hashlib
 import json
 import os
 import re
+import socket
 import statistics
 import subprocess
 import sys
@@ -44,22 +49,30 @@ from grouped_gemm_moesq_b200.metrics import packed_weight_bytes  # noqa: E402
 
 METRIC = "paired-4:8 NVFP4 grouped GEMM TFLOP/s + weight GB/s vs roofline, per token count"
 
-# name -> (E, k, H, I, T, routing, kind); kind "layer" or "gemm" (route + quantise + gate_up GEMM)
+KIMI = (384, 8, 7168, 2048)        # experts, top-k, hidden, intermediate
+LAYER_T = (1, 16, 64, 256, 1024, 4096, 16384)
+
+# name -> (E, k, H, I, T, routing, kind).  kind: "layer" (the whole path),
+# "gemm" (route + quantise + gate_up GEMM), "gemm_down" (route + quantise +
+# down GEMM), "quant_gemm" (fixed grouping, routed once outside the step:
+# activation quantisation + gate_up GEMM, as the paper's kernel benchmark),
+# "quant_gemm_down" (the same with the down shape).
 WORKLOADS = {
     "30b_layer_t256": (128, 8, 2048, 768, 256, "uniform", "layer"),
     "tiny_layer_t64": (8, 2, 512, 256, 64, "uniform", "layer"),
-    "kimi_layer_t1": (384, 8, 7168, 2048, 1, "uniform", "layer"),
-    "kimi_layer_t16": (384, 8, 7168, 2048, 16, "uniform", "layer"),
-    "kimi_layer_t64": (384, 8, 7168, 2048, 64, "uniform", "layer"),
-    "kimi_layer_t256": (384, 8, 7168, 2048, 256, "uniform", "layer"),
-    "kimi_layer_t4096_zipf": (384, 8, 7168, 2048, 4096, "zipf", "layer"),
-    "kimi_gateup_t1": (384, 8, 7168, 2048, 1, "uniform", "gemm"),
-    "kimi_gateup_t16": (384, 8, 7168, 2048, 16, "uniform", "gemm"),
-    "kimi_gateup_t64": (384, 8, 7168, 2048, 64, "uniform", "gemm"),
-    "kimi_gateup_t256": (384, 8, 7168, 2048, 256, "uniform", "gemm"),
-    "kimi_down_t8192_zipf": (384, 8, 7168, 2048, 8192, "zipf", "gemm_down"),
+    "kimi_gateup_t1": KIMI + (1, "uniform", "gemm"),
+    "kimi_gateup_t16": KIMI + (16, "uniform", "gemm"),
+    "kimi_gateup_t64": KIMI + (64, "uniform", "gemm"),
+    "kimi_gateup_t256": KIMI + (256, "uniform", "gemm"),
+    "kimi_down_t8192_zipf": KIMI + (8192, "zipf", "gemm_down"),
     "30b_gateup_t256": (128, 8, 2048, 768, 256, "uniform", "gemm"),
+    # compute-bound probes: 32 experts of the Kimi shapes, 4096 rows each
+    "cb_gateup_e32_n4096": (32, 8, 7168, 2048, 16384, "fixed4096", "quant_gemm"),
+    "cb_down_e32_n4096": (32, 8, 7168, 2048, 16384, "fixed4096", "quant_gemm_down"),
 }
+for _t in LAYER_T:
+    WORKLOADS["kimi_layer_t%d" % _t] = KIMI + (_t, "uniform", "layer")
+    WORKLOADS["kimi_layer_t%d_zipf" % _t] = KIMI + (_t, "zipf", "layer")
 # The paper's Table 11 setting (App. D, B200): Kimi gate_up over all 384
 # experts, expert g receiving N * {1, 3/4, 1/2, 1/4}[g % 4] rows, timed as
 # activation quantisation + grouped GEMM (bf16 in, bf16 out); the step is
@@ -68,9 +81,16 @@ WORKLOADS = {
 TAB11 = {8: (760.0, 148.0), 16: (793.0, 284.0), 32: (843.0, 535.0), 64: (925.0, 975.0),
          128: (912.0, 1978.0), 256: (1370.0, 2633.0)}
 for _n in TAB11:
-    WORKLOADS["tab11_n%d" % _n] = (384, 8, 7168, 2048, 30 * _n, "tab11", "quant_gemm")
-DEFAULT_WORKLOAD = "30b_layer_t256"
+    WORKLOADS["tab11_n%d" % _n] = KIMI + (30 * _n, "tab11", "quant_gemm")
 
+# Sweeps: one JSON line whose headline is one point and whose `sweep` holds
+# every point (all share the packed weights).
+SWEEPS = {
+    "kimi_layer": {"points": ["kimi_layer_t%d%s" % (t, r) for t in LAYER_T for r in ("", "_zipf")],
+                   "headline": "kimi_layer_t4096_zipf"},
+    "tab11": {"points": ["tab11_n%d" % n for n in TAB11], "headline": "tab11_n64"},
+}
+DEFAULT_WORKLOAD = "kimi_layer"
 
 FP4_OVER_BF16 = 4.0    # nominal dense tensor-core ratio, fp4 : bf16 (9 : 2.25 PFLOP/s)
 SPARSE_FACTOR = 2.0    # a structured-sparse MMA runs the dense-equivalent contraction at twice the rate
@@ -140,8 +160,28 @@ def gemm_roofline(gbytes, gfl, gemm_ms, peaks, traffic, gname):
     return roofline
 
 
+def host_cpu():
+    """Host threads available to this process and the CPU model."""
+    model = "unknown"
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                model = ln.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    try:
+        nproc = len(os.sched_getaffinity(0))
+    except AttributeError:
+        nproc = os.cpu_count()
+    return nproc, model
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
+    """nvidia-smi samples of one GPU's clocks and throttle reasons while
+    sampling is on; start/stop may be called repeatedly (one window per
+    timed region) and `summary` covers all windows."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -150,6 +190,8 @@ class ClockSampler:
         self.idx = device_index
         self.proc = None
         self.path = None
+        self.rows = []
+        self.ok = True
 
     def start(self):
         try:
@@ -161,21 +203,25 @@ class ClockSampler:
                                          stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+            self.ok = False
 
     def stop(self):
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+            return
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-        rows = []
         for line in open(self.path):
             parts = [p.strip() for p in line.split(",")]
             if len(parts) >= 9:
-                rows.append(parts)
+                self.rows.append(parts)
         os.unlink(self.path)
+        self.proc = None
+
+    def summary(self):
+        rows = self.rows
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
         sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
@@ -188,12 +234,17 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ work accounting
+def main_gemm_shape(kind, H, I):
+    """(M, K) of the workload's main grouped GEMM."""
+    return (H, I) if kind in ("gemm_down", "quant_gemm_down") else (2 * I, H)
+
+
 def step_work(E, k, H, I, T, counts_gu, kind):
     """(flops, weight bytes, per-GEMM algorithmic bytes, per-GEMM dense-equivalent
     flops) of one step."""
-    R = T * k
+    R = int(np.asarray(counts_gu).sum()) if kind.startswith("quant_gemm") else T * k
     touched = int((np.asarray(counts_gu) > 0).sum())
-    if kind == "gemm_down":
+    if kind in ("gemm_down", "quant_gemm_down"):
         M, K = H, I
         flops = 2.0 * M * K * R
         wbytes = touched * packed_weight_bytes(M, K)
@@ -207,6 +258,14 @@ def step_work(E, k, H, I, T, counts_gu, kind):
     dn_bytes = dn_w + R * (I // 2 + I // 32) + R * H * 2
     dn_fl = 2.0 * H * I * R
     return gu_fl + dn_fl, gu_w + dn_w, {"gate_up": gu_bytes, "down": dn_bytes}, {"gate_up": gu_fl, "down": dn_fl}
+
+
+def launches_per_step(kind, T):
+    """Kernels of this library one step launches: routing is top-k plus one
+    finishing kernel for T <= 512 tokens, else top-k, count, scan, scatter;
+    then quantise and the GEMM, and for the layer SwiGLU, down GEMM, combine."""
+    route = 0 if kind.startswith("quant_gemm") else (2 if T <= 512 else 4)
+    return route + 2 + (3 if kind == "layer" else 0)
 
 
 def rank_seed(seed, rank):
@@ -232,12 +291,12 @@ def job_throughput(flops_per_rank, world, ms):
     return world * flops_per_rank / (ms * 1e-3) / 1e12
 
 
-def tab11_logits(T, E, k=8):
-    """0/1 router logits whose top-k gives expert g exactly
-    N * {4, 3, 2, 1}[g % 4] / 4 rows (N = T / 30): every token takes the k
-    experts with the most rows still to fill (ties to the lower id)."""
-    n = T // 30
-    left = np.array([n * (4 - g % 4) // 4 for g in range(E)], np.int64)
+def fixed_count_logits(T, want, k=8):
+    """0/1 router logits [T, E] whose top-k gives expert g exactly want[g]
+    rows (sum(want) = T * k): every token takes the k experts with the most
+    rows still to fill (ties to the lower id)."""
+    left = np.array(want, np.int64)
+    E = left.size
     assert left.sum() == T * k
     lg = np.zeros((T, E), np.float32)
     for t in range(T):
@@ -248,237 +307,284 @@ def tab11_logits(T, E, k=8):
     return lg
 
 
+def tab11_logits(T, E, k=8):
+    """The Table 11 pattern: expert g gets N * {4, 3, 2, 1}[g % 4] / 4 rows,
+    N = T / 30."""
+    n = T // 30
+    return fixed_count_logits(T, [n * (4 - g % 4) // 4 for g in range(E)], k)
+
+
 def logits_for(routing, seed, T, E):
     if routing == "tab11":
         return tab11_logits(T, E)
+    if routing.startswith("fixed"):
+        n = int(routing[len("fixed"):])
+        return fixed_count_logits(T, [n] * E)
     return S.zipf_logits_np(seed, T, E) if routing == "zipf" else S.uniform_logits_np(seed, T, E)
+
+
+def workload_points(name):
+    """(points, headline) of a workload name: a sweep or a single workload."""
+    if name in SWEEPS:
+        return list(SWEEPS[name]["points"]), SWEEPS[name]["headline"]
+    return [name], name
 
 
 # ------------------------------------------------------------------ CUDA arm
 def run_cuda(args, rank, world, local_rank):
+    """Times every point of the workload on this rank's GPU.  Returns
+    {"points": {name: point}, "headline": name, "clocks": {...}}."""
     import torch
     import grouped_gemm_moesq_b200 as m
     from grouped_gemm_moesq_b200 import build as cuda_build
+    from cuda.bindings import runtime as cudart
 
     if rank == 0 or not os.path.exists(cuda_build.LIB):
         cuda_build.build()
     m.load()
     torch.cuda.set_device(local_rank)
     dev = "cuda"
-    E, k, H, I, T, routing, kind = WORKLOADS[args.workload]
     seed = 1234
     stream = torch.cuda.current_stream()
-
-    # weights: drawn on the GPU (same bits as the host generator) and packed, 8 experts at a time
-    def make_weights(linear, M, K):
-        pw = m.PackedWeights(E, M, K)
-        for e0 in range(0, E, 8):
-            n = min(8, E - e0)
-            w = torch.stack([S.expert_weights_bf16_torch(seed, linear, e, M, K, dev) for e in range(e0, e0 + n)])
-            m.moesq_pack_weights(w, e0, n, pw)
-            del w
-        return pw
-
-    if kind == "gemm_down":
-        w_main = make_weights(1, H, I)
-        w_dn = None
-    else:
-        w_main = make_weights(0, 2 * I, H)
-        w_dn = make_weights(1, H, I) if kind == "layer" else None
-    torch.cuda.synchronize()
-
-    # per-rank batch (independent replicas: weak scaling, no data-path collective)
-    K_in = I if kind == "gemm_down" else H
-    x_np = S.activations_bf16_np(rank_seed(seed, rank), T, K_in)
-    lg_np = logits_for(routing, rank_seed(seed, rank), T, E)
-    x = torch.from_numpy(x_np.view(np.int16).copy()).to(dev).view(torch.bfloat16)
-    lg = torch.from_numpy(lg_np).to(dev)
-
-    rb = m.RoutingBuffers(T, E, k)
-    ga = torch.empty(E, dtype=torch.float32, device=dev)
-    gh = torch.empty(E, dtype=torch.float32, device=dev)
-    if kind == "layer":
-        ws = torch.empty(m.moesq_layer_workspace_bytes(T, k, E, H, I), dtype=torch.uint8, device=dev)
-        m.moesq_calibrate_layer(x, lg, T, k, w_main, w_dn, ga, gh, ws)
-    else:
-        m.moesq_act_global_scale(x, ga[:1])
-        ga.fill_(float(ga[:1].item()))
-    a_codes, a_scales = m.act_buffers(rb.rows_cap, K_in)
-    M_main = w_main.M
-    y_main = torch.empty(rb.rows_cap, M_main, dtype=torch.bfloat16, device=dev)
-    if kind == "layer":
-        h_codes, h_scales = m.act_buffers(rb.rows_cap, I)
-        y_dn = torch.empty(rb.rows_cap, H, dtype=torch.bfloat16, device=dev)
-        out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
-
-    # the hot path as its ABI calls, one callable per component
-    def c_route_quant():
-        m.moesq_route_permute(lg, rb)
-        m.moesq_quantize_act(x, T, K_in, rb, ga, rb.rows_cap, a_codes, a_scales)
-
-    # GEMM configurations, frozen by moesq_gemm_autotune after the warm-up
-    # and before the graphs are captured
-    tuned = {"main": (0, 0), "down": (0, 0)}
-
-    def c_gemm_main():
-        tn, nc = tuned["main"]
-        m.moesq_grouped_sparse_gemm(w_main, a_codes, a_scales, rb.rows_cap, rb.counts, rb.row_offsets, ga, y_main,
-                                    tile_n=tn, num_ctas=nc)
-
-    if kind == "quant_gemm":                  # fixed grouping: routed once, outside the step
-        m.moesq_route_permute(lg, rb)
-        comps = [("quant", lambda: m.moesq_quantize_act(x, T, K_in, rb, ga, rb.rows_cap, a_codes, a_scales)),
-                 ("gemm_main", c_gemm_main)]
-    else:
-        comps = [("route_quant", c_route_quant), ("gemm_main", c_gemm_main)]
-    if kind == "layer":
-        comps += [("swiglu_quant", lambda: m.moesq_swiglu_quant(y_main, I, rb, gh, h_codes, h_scales)),
-                  ("gemm_down", lambda: m.moesq_grouped_sparse_gemm(w_dn, h_codes, h_scales, rb.rows_cap, rb.counts,
-                                                                    rb.row_offsets, gh, y_dn, tile_n=tuned["down"][0],
-                                                                    num_ctas=tuned["down"][1])),
-                  ("combine", lambda: m.moesq_combine(y_dn, H, rb, out))]
-
-    def step_eager():
-        for _, f in comps:
-            f()
-
-    # routing: top-k plus one finishing kernel for T <= 512 tokens, else top-k, count, scan and scatter
-    launches_per_step = (0 if kind == "quant_gemm" else 2 if T <= 512 else 4) + 2 + (3 if kind == "layer" else 0)
+    points, headline = workload_points(args.workload)
+    clocks = ClockSampler(local_rank)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    for _ in range(args.warmup):
-        flush.zero_()
-        step_eager()
-    torch.cuda.synchronize()
-    st, word = m.moesq_get_device_error()
-    if st != 0:
-        raise RuntimeError("device error word %#x during warm-up" % word)
-    tuned["main"] = m.moesq_gemm_autotune(w_main, a_codes, a_scales, rb.rows_cap, rb.counts, rb.row_offsets, ga,
-                                          y_main, reps=3)[0]
-    if kind == "layer":
-        tuned["down"] = m.moesq_gemm_autotune(w_dn, h_codes, h_scales, rb.rows_cap, rb.counts, rb.row_offsets, gh,
-                                              y_dn, reps=3)[0]
-    step_eager()                              # outputs of the tuned configuration
-    torch.cuda.synchronize()
-    counts = rb.counts.cpu().numpy()
 
-    # One CUDA graph per step (the pages time CUDA-graph replays, App. D.2),
-    # with external event-record nodes between the components: the same
-    # replays give the per-kernel breakdown on the launching stream.
-    from cuda.bindings import runtime as cudart
+    # packed weights, drawn on the GPU (same bits as the host generator) and
+    # packed 8 experts at a time; shared by every point with the same shapes
+    wcache = {}
+
+    def weights(linear, E, M, K):
+        key = (linear, E, M, K)
+        if key not in wcache:
+            pw = m.PackedWeights(E, M, K)
+            for e0 in range(0, E, 8):
+                n = min(8, E - e0)
+                w = torch.stack([S.expert_weights_bf16_torch(seed, linear, e, M, K, dev) for e in range(e0, e0 + n)])
+                m.moesq_pack_weights(w, e0, n, pw)
+                del w
+            torch.cuda.synchronize()
+            wcache[key] = pw
+        return wcache[key]
 
     def cu_event():
         err, e = cudart.cudaEventCreate()
         assert err == cudart.cudaError_t.cudaSuccess
         return e
 
-    cev = [cu_event() for _ in range(len(comps) + 1)]
-    g_step = torch.cuda.CUDAGraph()          # the timed step: kernels only
-    with torch.cuda.graph(g_step):
-        step_eager()
-    g_prof = torch.cuda.CUDAGraph()          # the same kernels with event nodes between them
-    with torch.cuda.graph(g_prof):
-        cs = torch.cuda.current_stream().cuda_stream
-        for j, (_, f) in enumerate(comps):
-            cudart.cudaEventRecordWithFlags(cev[j], cs, cudart.cudaEventRecordExternal)
-            f()
-        cudart.cudaEventRecordWithFlags(cev[-1], cs, cudart.cudaEventRecordExternal)
-    flush.zero_()
-    g_step.replay()
-    g_prof.replay()
-    torch.cuda.synchronize()
+    # this GPU's measured ceiling for the MMA the GEMM issues (no memory traffic)
+    fp4_peak = {"sparse_n256_1cta": m.moesq_mma_peak(1, 256, 1), "sparse_n128_2cta": m.moesq_mma_peak(1, 128, 2),
+                "dense_n256_1cta": m.moesq_mma_peak(0, 256, 1),
+                "sparse_n128_2cta_with_scale_copies": m.moesq_mma_peak(1, 128, 2, with_copies=True)}
 
-    def ev():
-        return torch.cuda.Event(enable_timing=True)
+    results = {}
+    for name in points:
+        E, k, H, I, T, routing, kind = WORKLOADS[name]
+        down_main = kind in ("gemm_down", "quant_gemm_down")
+        if down_main:
+            w_main, w_dn = weights(1, E, H, I), None
+        else:
+            w_main = weights(0, E, 2 * I, H)
+            w_dn = weights(1, E, H, I) if kind == "layer" else None
 
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-    torch.cuda.synchronize()
-    clocks = ClockSampler(local_rank)
-    clocks.start()
-    time.sleep(0.3)
-    t_wall0 = time.perf_counter()
-    evs = [(ev(), ev()) for _ in range(args.steps)]
-    part_ms = {name: [] for name, _ in comps}
-    for i in range(args.steps):
+        # this rank's batch (independent replicas: weak scaling, no data-path collective)
+        K_in = I if down_main else H
+        x = S.activations_bf16_torch(rank_seed(seed, rank), T, K_in, dev)
+        lg_np = logits_for(routing, rank_seed(seed, rank), T, E)
+        lg = torch.from_numpy(lg_np).to(dev)
+        rb = m.RoutingBuffers(T, E, k)
+        ga = torch.empty(E, dtype=torch.float32, device=dev)
+        gh = torch.empty(E, dtype=torch.float32, device=dev)
+        if kind == "layer":
+            ws = torch.empty(m.moesq_layer_workspace_bytes(T, k, E, H, I), dtype=torch.uint8, device=dev)
+            m.moesq_calibrate_layer(x, lg, T, k, w_main, w_dn, ga, gh, ws)
+            del ws
+        else:
+            m.moesq_act_global_scale(x, ga[:1])
+            ga.fill_(float(ga[:1].item()))
+        a_codes, a_scales = m.act_buffers(rb.rows_cap, K_in)
+        y_main = torch.empty(rb.rows_cap, w_main.M, dtype=torch.bfloat16, device=dev)
+        if kind == "layer":
+            h_codes, h_scales = m.act_buffers(rb.rows_cap, I)
+            y_dn = torch.empty(rb.rows_cap, H, dtype=torch.bfloat16, device=dev)
+            out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+
+        # GEMM configurations, frozen by moesq_gemm_autotune after the warm-up
+        # and before the graphs are captured
+        tuned = {"main": (0, 0, 0), "down": (0, 0, 0)}
+
+        def c_route_quant():
+            m.moesq_route_permute(lg, rb)
+            m.moesq_quantize_act(x, T, K_in, rb, ga, rb.rows_cap, a_codes, a_scales)
+
+        def c_gemm_main():
+            tn, nc, cps = tuned["main"]
+            m.moesq_grouped_sparse_gemm(w_main, a_codes, a_scales, rb.rows_cap, rb.counts, rb.row_offsets, ga,
+                                        y_main, tile_n=tn, num_ctas=nc, sm_mode=cps)
+
+        if kind.startswith("quant_gemm"):     # fixed grouping: routed once, outside the step
+            m.moesq_route_permute(lg, rb)
+            comps = [("quant", lambda: m.moesq_quantize_act(x, T, K_in, rb, ga, rb.rows_cap, a_codes, a_scales)),
+                     ("gemm_main", c_gemm_main)]
+        else:
+            comps = [("route_quant", c_route_quant), ("gemm_main", c_gemm_main)]
+        if kind == "layer":
+            comps += [("swiglu_quant", lambda: m.moesq_swiglu_quant(y_main, I, rb, gh, h_codes, h_scales)),
+                      ("gemm_down", lambda: m.moesq_grouped_sparse_gemm(
+                          w_dn, h_codes, h_scales, rb.rows_cap, rb.counts, rb.row_offsets, gh, y_dn,
+                          tile_n=tuned["down"][0], num_ctas=tuned["down"][1], sm_mode=tuned["down"][2])),
+                      ("combine", lambda: m.moesq_combine(y_dn, H, rb, out))]
+
+        def step_eager():
+            for _, f in comps:
+                f()
+
+        for _ in range(args.warmup):
+            flush.zero_()
+            step_eager()
+        torch.cuda.synchronize()
+        st, word = m.moesq_get_device_error()
+        if st != 0:
+            raise RuntimeError("%s: device error word %#x during warm-up" % (name, word))
+        tuned["main"] = m.moesq_gemm_autotune(w_main, a_codes, a_scales, rb.rows_cap, rb.counts, rb.row_offsets,
+                                              ga, y_main, reps=3)[0]
+        if kind == "layer":
+            tuned["down"] = m.moesq_gemm_autotune(w_dn, h_codes, h_scales, rb.rows_cap, rb.counts,
+                                                  rb.row_offsets, gh, y_dn, reps=3)[0]
+        step_eager()                          # outputs of the tuned configuration
+        torch.cuda.synchronize()
+        counts = rb.counts.cpu().numpy()
+
+        # One CUDA graph per step (the pages time CUDA-graph replays, App. D.2),
+        # and a second one with external event-record nodes between the
+        # components: the same replays give the per-kernel breakdown on the
+        # launching stream.
+        cev = [cu_event() for _ in range(len(comps) + 1)]
+        g_step = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_step):
+            step_eager()
+        g_prof = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_prof):
+            cs = torch.cuda.current_stream().cuda_stream
+            for j, (_, f) in enumerate(comps):
+                cudart.cudaEventRecordWithFlags(cev[j], cs, cudart.cudaEventRecordExternal)
+                f()
+            cudart.cudaEventRecordWithFlags(cev[-1], cs, cudart.cudaEventRecordExternal)
         flush.zero_()
-        evs[i][0].record(stream)
         g_step.replay()
-        evs[i][1].record(stream)
-    torch.cuda.synchronize()
-    t_wall = time.perf_counter() - t_wall0
-    for i in range(args.steps):                 # per-kernel breakdown, same flush discipline
-        flush.zero_()
         g_prof.replay()
         torch.cuda.synchronize()
-        for j, (name, _) in enumerate(comps):
-            err, dt = cudart.cudaEventElapsedTime(cev[j], cev[j + 1])
-            assert err == cudart.cudaError_t.cudaSuccess, err
-            part_ms[name].append(dt)
-    if world > 1:
-        dist.barrier()
-    clk = clocks.stop()
-    st, word = m.moesq_get_device_error()
-    if st != 0:
-        raise RuntimeError("device error word %#x in the timed region" % word)
 
-    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
-    parts = {name: statistics.mean(v) for name, v in part_ms.items()}
-    del g_step, g_prof
-    for e in cev:
-        cudart.cudaEventDestroy(e)
-
-    # e2e through the public host-buffer entry point (layer workloads)
-    e2e = None
-    if kind == "layer":
-        wsh = torch.empty(m.moesq_layer_host_workspace_bytes(T, k, E, H, I), dtype=torch.uint8, device=dev)
-        xh = torch.from_numpy(x_np.view(np.int16).copy()).pin_memory()
-        lh = torch.from_numpy(lg_np).pin_memory()
-        oh = torch.empty(T, H, dtype=torch.int16).pin_memory()
-        for _ in range(args.warmup):
-            m.moesq_moe_layer_host(xh, lh, T, k, w_main, w_dn, ga, gh, oh, wsh)
-        e2e_ms = []
-        for _ in range(args.steps):
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize()
+        clocks.start()
+        time.sleep(0.2)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        for i in range(args.steps):
             flush.zero_()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            m.moesq_moe_layer_host(xh, lh, T, k, w_main, w_dn, ga, gh, oh, wsh)
-            b.record(stream)
-            b.synchronize()
-            e2e_ms.append(a.elapsed_time(b))
-        e2e = {"ms_per_step": statistics.mean(e2e_ms),
-               "h2d_bytes_per_step": T * H * 2 + T * E * 4, "d2h_bytes_per_step": T * H * 2}
+            evs[i][0].record(stream)
+            g_step.replay()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        clocks.stop()
+        part_ms = {pname: [] for pname, _ in comps}
+        for i in range(args.steps):             # per-kernel breakdown, same flush discipline
+            flush.zero_()
+            g_prof.replay()
+            torch.cuda.synchronize()
+            for j, (pname, _) in enumerate(comps):
+                err, dt = cudart.cudaEventElapsedTime(cev[j], cev[j + 1])
+                assert err == cudart.cudaError_t.cudaSuccess, err
+                part_ms[pname].append(dt)
+        st, word = m.moesq_get_device_error()
+        if st != 0:
+            raise RuntimeError("%s: device error word %#x in the timed region" % (name, word))
+        ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+        parts = {pname: statistics.mean(v) for pname, v in part_ms.items()}
+        del g_step, g_prof
+        for e in cev:
+            cudart.cudaEventDestroy(e)
 
-    flops, wbytes, gemm_bytes, gemm_fl = step_work(E, k, H, I, T, counts, kind)
-    t_max, e2e_max = max_over_ranks([ms, e2e["ms_per_step"] if e2e else 0.0], device=dev)
-    if e2e:
-        e2e["ms_per_step"] = e2e_max
-    return dict(kind=kind, E=E, k=k, H=H, I=I, T=T, routing=routing, ms=t_max, parts=parts, flops=flops,
-                wbytes=wbytes, gemm_bytes=gemm_bytes, gemm_fl=gemm_fl, e2e=e2e, tuned=tuned, clocks=clk, launches=launches_per_step * args.steps,
-                wall_s=t_wall, counts=counts)
+        # e2e through the public host-buffer entry point (layer workloads):
+        # pinned host input and logits in, output back, inside the timed region
+        e2e = None
+        if kind == "layer":
+            wsh = torch.empty(m.moesq_layer_host_workspace_bytes(T, k, E, H, I), dtype=torch.uint8, device=dev)
+            xh = x.view(torch.int16).cpu().pin_memory()
+            lh = torch.from_numpy(lg_np).pin_memory()
+            oh = torch.empty(T, H, dtype=torch.int16).pin_memory()
+            for _ in range(args.warmup):
+                m.moesq_moe_layer_host(xh, lh, T, k, w_main, w_dn, ga, gh, oh, wsh)
+            e2e_ms = []
+            for _ in range(args.steps):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                m.moesq_moe_layer_host(xh, lh, T, k, w_main, w_dn, ga, gh, oh, wsh)
+                b.record(stream)
+                b.synchronize()
+                e2e_ms.append(a.elapsed_time(b))
+            e2e = {"ms_per_step": statistics.mean(e2e_ms),
+                   "h2d_bytes_per_step": T * H * 2 + T * E * 4, "d2h_bytes_per_step": T * H * 2}
+            del wsh, xh, lh, oh
+
+        flops, wbytes, gemm_bytes, gemm_fl = step_work(E, k, H, I, T, counts, kind)
+        t_max, e2e_max = max_over_ranks([ms, e2e["ms_per_step"] if e2e else 0.0], device=dev)
+        if e2e:
+            e2e["ms_per_step"] = e2e_max
+        results[name] = dict(kind=kind, E=E, k=k, H=H, I=I, T=T, routing=routing, ms=t_max, parts=parts,
+                             flops=flops, wbytes=wbytes, gemm_bytes=gemm_bytes, gemm_fl=gemm_fl, e2e=e2e,
+                             tuned=dict(tuned), launches=launches_per_step(kind, T), counts=counts)
+        del x, lg, rb, a_codes, a_scales, y_main
+        if kind == "layer":
+            del h_codes, h_scales, y_dn, out
+        torch.cuda.empty_cache()
+    return {"points": results, "headline": headline, "clocks": clocks.summary(), "fp4_peak": fp4_peak}
 
 
 # ------------------------------------------------------------------ oracle (CPU) arm
 _ORACLE_PREP = {}
 
 
+def _host_weights(seed, linear, e, M, K):
+    """One expert's seeded bf16 weight bits: drawn by the generator's torch
+    path on a GPU when one is present (seconds less per Kimi expert), else on
+    the host; the bits are the same."""
+    try:
+        import torch
+        if torch.cuda.is_available():
+            w = S.expert_weights_bf16_torch(seed, linear, int(e), M, K, "cuda")
+            return w.view(torch.int16).cpu().numpy().view(np.uint16)
+    except ImportError:
+        pass
+    return S.expert_weights_bf16_np(seed, linear, int(e), M, K)
+
+
 def oracle_prepare(workload, n_tokens, seed=1234):
-    """Inputs, routing and packed weights (the touched experts only) of the
-    first n_tokens tokens of the workload's batch; made once per run, outside
-    every timed region."""
+    """Inputs, routing, packed weights (the touched experts only) and the
+    activation global scales of the first n_tokens tokens of the workload's
+    batch; made once per run, outside every timed region.  For the layer the
+    global scales are the oracle's own calibration on that sample."""
     key = (workload, n_tokens, seed)
     if key in _ORACLE_PREP:
         return _ORACLE_PREP[key]
     import oracle as O
     E, k, H, I, T, routing, kind = WORKLOADS[workload]
     n = min(n_tokens, T)
-    K_in = I if kind == "gemm_down" else H
+    down_main = kind in ("gemm_down", "quant_gemm_down")
+    K_in = I if down_main else H
     x = S.activations_bf16_np(seed, T, K_in, rows=n)
     lg = logits_for(routing, seed, T, E)[:n]
     used = np.nonzero(O.route(lg, k).counts)[0]
 
     def packed(linear, M, K):
-        w = np.stack([S.expert_weights_bf16_np(seed, linear, int(e), M, K) for e in used])
+        w = np.stack([_host_weights(seed, linear, e, M, K) for e in used])
         pk = O.pack_weights(w)
         full = O.Packed(np.zeros((E, M, K // 4), np.uint8), np.zeros((E, M, K // 16), np.uint8),
                         np.zeros((E, M, K // 32), np.uint8), np.ones(E, np.float32))
@@ -487,8 +593,8 @@ def oracle_prepare(workload, n_tokens, seed=1234):
         return full
 
     prep = {"n": n, "x": x, "lg": lg, "k": k, "kind": kind,
-            "ga": np.full(E, O.act_global_scale(x), np.float32), "gh": np.full(E, 64.0, np.float32)}
-    if kind == "gemm_down":
+            "ga": np.full(E, O.act_global_scale(x), np.float32)}
+    if down_main:
         prep["pk"] = packed(1, H, I)
         prep["flops"] = 2.0 * H * I * n * k
     else:
@@ -497,13 +603,15 @@ def oracle_prepare(workload, n_tokens, seed=1234):
         if kind == "layer":
             prep["pk_dn"] = packed(1, H, I)
             prep["flops"] = 2.0 * 3 * I * H * n * k
+            prep["ga"], prep["gh"] = O.calibrate_layer(x, lg, k, prep["pk"], prep["pk_dn"])
     _ORACLE_PREP[key] = prep
     return prep
 
 
 def run_oracle_sample(workload, n_tokens, seed=1234):
     """Times one pass of the oracle over the prepared token sample (routing,
-    quantisation and the GEMMs, or the whole layer).  Returns (seconds, flops)."""
+    quantisation and the GEMM(s), or the whole layer).  Returns (seconds,
+    dense-equivalent flops)."""
     import oracle as O
     p = oracle_prepare(workload, n_tokens, seed)
     t0 = time.perf_counter()
@@ -533,52 +641,102 @@ def oracle_sample_tokens(workload):
     few enough touched experts (about 150 M weights to draw and pack) that
     the preparation stays under a minute or so."""
     E, k, H, I, T, routing, kind = WORKLOADS[workload]
-    per_token_macs = k * (3 * I * H if kind == "layer" else 2 * I * H if kind in ("gemm", "quant_gemm") else H * I)
-    weights_per_expert = 3 * I * H if kind == "layer" else 2 * I * H if kind in ("gemm", "quant_gemm") else H * I
-    by_macs = int(2.5e9 // per_token_macs)
-    by_prep = int(150e6 // (k * weights_per_expert))
+    per_expert = 3 * I * H if kind == "layer" else H * I if kind in ("gemm_down", "quant_gemm_down") else 2 * I * H
+    by_macs = int(2.5e9 // (k * per_expert))
+    by_prep = int(150e6 // (k * per_expert))
     return max(1, min(T, by_macs, by_prep))
 
 
+def cpu_baseline_record(value, n, T, passes, secs, what):
+    nproc, model = host_cpu()
+    return {"value": value, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+            "sample": "first %d of %d tokens of %s, %d passes (%.1f s), one host thread" % (n, T, what, passes, secs),
+            "host_threads_available": nproc, "cpu_model": model}
+
+
 # ------------------------------------------------------------------ main
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def launch_ranks(n):
+    """Re-runs this script as n ranks under torch.distributed.run on this
+    node (one process per GPU, rendezvous on 127.0.0.1), bounded by timeout;
+    returns the launcher's exit code."""
+    cmd = ["timeout", "-k", "60", "3600", sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           "--nproc-per-node", str(n), "--master-addr", "127.0.0.1", "--master-port", str(_free_port()),
+           os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
+def point_entry(name, r, peaks):
+    """One sweep entry: the point's step time, throughput and GEMM fractions."""
+    ent = {"workload": name, "tokens": r["T"], "routing": r["routing"], "ms_per_step": r["ms"],
+           "tflops": r["flops"] / (r["ms"] * 1e-3) / 1e12,
+           "weight_gbs": r["wbytes"] / (r["ms"] * 1e-3) / 1e9, "breakdown_ms": r["parts"],
+           "expert_rows": {"min": int(r["counts"].min()), "max": int(r["counts"].max()),
+                           "touched": int((r["counts"] > 0).sum())},
+           "gemm_config": {g: {"tile_n": tn, "num_ctas": nc, "sm_mode": cps}
+                           for g, (tn, nc, cps) in r["tuned"].items() if tn}}
+    gemms = {}
+    for gname, part in (("gate_up", "gemm_main"), ("down", "gemm_down" if r["kind"] == "layer" else "gemm_main")):
+        if gname in r["gemm_bytes"] and part in r["parts"]:
+            rf = gemm_roofline(r["gemm_bytes"][gname], r["gemm_fl"][gname], r["parts"][part], peaks, None, gname)
+            gemms[gname] = {"ms": r["parts"][part], "hbm_frac": rf["hbm_frac"], "tensor_frac": rf["tensor_frac"],
+                            "bound": rf["bound"], "frac": rf["frac"]}
+    ent["gemms"] = gemms
+    if r["e2e"]:
+        ent["e2e_ms"] = r["e2e"]["ms_per_step"]
+        ent["e2e_tflops"] = r["flops"] / (r["e2e"]["ms_per_step"] * 1e-3) / 1e12
+    return ent
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--gpus", type=int, default=None)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(set(WORKLOADS) | set(SWEEPS)))
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
 
+    if "WORLD_SIZE" not in os.environ and args.gpus is not None and args.gpus > 1:
+        sys.exit(launch_ranks(args.gpus))
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    E, k, H, I, T, routing, kind = WORKLOADS[args.workload]
-    config = {"workload": args.workload, "experts": E, "top_k": k, "hidden": H, "intermediate": I,
-              "tokens_per_gpu": T, "routing": routing, "step": kind,
-              "l2": "flushed (256 MiB write) before every step, outside the timed events",
-              "timing": "CUDA-graph replay of the step, CUDA events on the launching stream"}
+    if args.gpus is not None and args.gpus != world:
+        raise SystemExit("--gpus %d but WORLD_SIZE=%d" % (args.gpus, world))
+    points, headline = workload_points(args.workload)
+    E, k, H, I, T, routing, kind = WORKLOADS[headline]
+    config = {"workload": args.workload, "headline": headline, "experts": E, "top_k": k, "hidden": H,
+              "intermediate": I, "tokens_per_gpu": T, "routing": routing, "step": kind}
 
     if args.impl == "reference":
         if rank != 0:
             return
-        n = oracle_sample_tokens(args.workload)
-        oracle_prepare(args.workload, n)        # inputs and packed weights, not timed
+        n = oracle_sample_tokens(headline)
+        oracle_prepare(headline, n)             # inputs and packed weights, not timed
         for _ in range(args.warmup):
-            run_oracle_sample(args.workload, n)
+            run_oracle_sample(headline, n)
         secs, fl = [], 0.0
         for _ in range(args.steps):
-            s, fl = run_oracle_sample(args.workload, n)
+            s, fl = run_oracle_sample(headline, n)
             secs.append(s)
         v = fl / statistics.mean(secs) / 1e12
-        cores = 1
-        line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        rconfig = dict(config, timing="host wall clock (time.perf_counter) around each oracle pass over the "
+                                      "token sample; one host thread",
+                       l2="n/a (CPU oracle; inputs resident in host memory)")
+        line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(secs),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-                "data": "synthetic", "config": config,
-                "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                                 "sample": "first %d of %d tokens of the workload per step" % (n, T)},
+                "data": "synthetic", "config": rconfig,
+                "cpu_baseline": cpu_baseline_record(v, n, T, args.steps, sum(secs), headline),
                 "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line))
         return
@@ -588,9 +746,9 @@ def main():
         import torch.distributed as dist
         from datetime import timedelta
         torch.cuda.set_device(local_rank)
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
 
-    r = run_cuda(args, rank, world, local_rank)
+    res = run_cuda(args, rank, world, local_rank)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
@@ -600,23 +758,33 @@ def main():
         return
 
     peaks = load_peaks()
+    r = res["points"][res["headline"]]
     ms = r["ms"]
     value = job_throughput(r["flops"], world, ms)
     weight_gbs = world * r["wbytes"] / (ms * 1e-3) / 1e9
-    gname = "down" if r["kind"] == "gemm_down" else "gate_up"
+    gname = "down" if r["kind"] in ("gemm_down", "quant_gemm_down") else "gate_up"
     gemm_ms = r["parts"]["gemm_main"]
     gbytes, gfl = r["gemm_bytes"][gname], r["gemm_fl"][gname]
-    roofline = gemm_roofline(gbytes, gfl, gemm_ms, peaks, profiled_traffic(args.workload, gname), gname)
-    tab11_n = T // 30 if args.workload.startswith("tab11_") else None
+    roofline = gemm_roofline(gbytes, gfl, gemm_ms, peaks, profiled_traffic(res["headline"], gname), gname)
+    if res.get("fp4_peak"):
+        mp = max(v for k_, v in res["fp4_peak"].items() if k_.startswith("sparse") and "copies" not in k_)
+        roofline["tensor_frac_of_measured_fp4"] = roofline["dense_equiv_flops"] / (gemm_ms * 1e-3) / 1e12 / mp
+        roofline["measured_fp4_sparse_peak"] = mp
+        roofline["peak_source"] += ("; measured sparse FP4 MMA peak %.0f TFLOP/s (moesq_mma_peak, back-to-back "
+                                    "tcgen05.mma.sp kind::mxf4nvf4 on every SM)" % mp)
+    tab11_n = r["T"] // 30 if res["headline"].startswith("tab11_") else None
     vs_baseline = value / TAB11[tab11_n][1] if tab11_n else None
+    config.update({"l2": "flushed (256 MiB write) before every step, outside the timed events",
+                   "timing": "CUDA-graph replay of the step, CUDA events on the launching stream"})
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": vs_baseline, "dtype": "nvfp4 (e2m1 x ue4m3 products, f32 accumulate, bf16 out)",
             "data": "synthetic (seeded; pages' shapes and distributions)", "config": config,
             "weight_gbs": weight_gbs, "breakdown_ms": r["parts"], "roofline": roofline,
-            "gemm_config": {name: {"tile_n": tn, "num_ctas": nc} for name, (tn, nc) in r["tuned"].items()
-                            if tn},
-            "clocks": r["clocks"], "gpu_launches": r["launches"],
+            "gemm_config": {g: {"tile_n": tn, "num_ctas": nc, "sm_mode": cps}
+                            for g, (tn, nc, cps) in r["tuned"].items() if tn},
+            "clocks": res["clocks"], "gpu_launches": r["launches"] * args.steps,
+            "fp4_mma_peak_tflops": res.get("fp4_peak"),
             "expert_rows": {"min": int(r["counts"].min()), "max": int(r["counts"].max()),
                             "touched": int((r["counts"] > 0).sum())}}
     if r["e2e"]:
@@ -624,11 +792,11 @@ def main():
         line["e2e"] = {"value": job_throughput(r["flops"], world, e["ms_per_step"]), "unit": "TFLOP/s",
                        "h2d_bytes_per_step": e["h2d_bytes_per_step"], "d2h_bytes_per_step": e["d2h_bytes_per_step"],
                        "ms_per_step": e["ms_per_step"]}
+    if len(res["points"]) > 1:
+        line["sweep"] = [point_entry(nm, res["points"][nm], peaks) for nm in points]
     if world == 1 and not args.no_cpu_baseline:
-        v, secs, passes, n = oracle_baseline(args.workload)
-        line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
-                                "sample": "first %d of %d tokens of the workload, %d passes (%.1f s)"
-                                % (n, T, passes, secs)}
+        v, secs, passes, n = oracle_baseline(res["headline"])
+        line["cpu_baseline"] = cpu_baseline_record(v, n, r["T"], passes, secs, res["headline"])
     print(json.dumps(line))
     if world > 1:
         dist.destroy_process_group()

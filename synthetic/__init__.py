@@ -208,3 +208,49 @@ def expert_weights_bf16_torch(seed: int, linear: int, e: int, M: int, K: int, de
                               sigma: float = 0.02):
     return normal_bf16_torch(expert_weight_key(seed, linear, e), (M, K), sigma, device)
 
+
+
+def _normal_f64_torch(key: int, start: int, count: int, device):
+    """Same values as `normal_f64_np`, as a torch float64 tensor on `device`."""
+    torch, g, m1, m2 = _torch_consts()
+    skey = key - (1 << 64) if key >= (1 << 63) else key
+    idx = torch.arange(start, start + count, dtype=torch.int64, device=device) * 6
+    s = torch.zeros(count, dtype=torch.int64, device=device)
+    for j in range(6):
+        z = (idx + (j + 1)) * g + skey
+        u = _mix64_torch(torch, z, m1, m2)
+        s += _srl(torch, u, 40)
+        s += _srl(torch, u, 16) & 0xFFFFFF
+        del z, u
+    del idx
+    return (s - 6 * (1 << 24)).to(torch.float64) * (2.0 ** -24)
+
+
+def _f32_to_bf16_torch(f):
+    """float32 tensor -> bf16 tensor with round-to-nearest-even on the bit
+    pattern (the same bits as `f32_to_bf16_bits_np`)."""
+    import torch
+    u32 = f.contiguous().view(torch.int32).to(torch.int64) & 0xFFFFFFFF
+    bits = ((u32 + ((u32 >> 16) & 1) + 0x7FFF) >> 16) & 0xFFFF
+    out = bits.to(torch.int32)
+    out = torch.where(out >= 32768, out - 65536, out).to(torch.int16)
+    return out.view(torch.bfloat16)
+
+
+def activations_bf16_torch(seed: int, T: int, K: int, device, n_outliers: int = 4,
+                           outlier_gain: float = 20.0, label: int = 0, chunk_rows: int = 2048):
+    """Same bits as `activations_bf16_np`, drawn on `device` (a bf16 tensor
+    [T, K]), `chunk_rows` rows at a time."""
+    import torch
+    key = stream_key(seed, 1, label)
+    ch = outlier_channels(stream_key(seed, 2, label), K, n_outliers) if n_outliers else None
+    out = torch.empty((T, K), dtype=torch.bfloat16, device=device)
+    for r0 in range(0, T, chunk_rows):
+        n = min(chunk_rows, T - r0)
+        v = _normal_f64_torch(key, r0 * K, n * K, device).reshape(n, K)
+        if ch is not None:
+            idx = torch.as_tensor(ch, device=device)
+            v[:, idx] *= outlier_gain
+        out[r0:r0 + n] = _f32_to_bf16_torch(v.to(torch.float32))
+        del v
+    return out

@@ -102,22 +102,30 @@ def test_traffic_record_needs_the_current_gemm_source():
 
 
 def test_bench_line_has_the_contract_keys(monkeypatch, capsys):
-    """bench.main() composes one JSON line with every key of the contract
-    (a stand-in for the CUDA run supplies the measured parts)."""
+    """bench.main() composes one JSON line with every key of the contract,
+    the headline point's numbers and one sweep entry per point (a stand-in
+    for the CUDA run supplies the measured parts)."""
     import json
     import sys
     import bench
-    E, k, H, I, T, routing, kind = bench.WORKLOADS[bench.DEFAULT_WORKLOAD]
-    counts = np.full(E, T * k // E)
-    flops, wbytes, gbytes, gfl = bench.step_work(E, k, H, I, T, counts, kind)
+    points, headline = bench.workload_points(bench.DEFAULT_WORKLOAD)
+    assert headline in points and len(points) == 14
+
+    def fake_point(name):
+        E, k, H, I, T, routing, kind = bench.WORKLOADS[name]
+        counts = np.full(E, max(1, T * k // E))
+        flops, wbytes, gbytes, gfl = bench.step_work(E, k, H, I, T, counts, kind)
+        return dict(kind=kind, E=E, k=k, H=H, I=I, T=T, routing=routing, ms=0.5,
+                    parts={"route_quant": 0.05, "gemm_main": 0.2, "swiglu_quant": 0.02, "gemm_down": 0.2,
+                           "combine": 0.03},
+                    flops=flops, wbytes=wbytes, gemm_bytes=gbytes, gemm_fl=gfl,
+                    e2e={"ms_per_step": 0.9, "h2d_bytes_per_step": 1, "d2h_bytes_per_step": 2},
+                    tuned={"main": (128, 296, 1), "down": (128, 296, 1)}, launches=bench.launches_per_step(kind, T),
+                    counts=counts)
 
     def fake_run(args, rank, world, local_rank):
-        return dict(kind=kind, E=E, k=k, H=H, I=I, T=T, routing=routing, ms=0.08, parts={"gemm_main": 0.036},
-                    flops=flops, wbytes=wbytes, gemm_bytes=gbytes, gemm_fl=gfl,
-                    e2e={"ms_per_step": 0.16, "h2d_bytes_per_step": 1, "d2h_bytes_per_step": 2},
-                    tuned={"main": (64, 296), "down": (64, 296)},
-                    clocks={"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}, launches=140, wall_s=0.01,
-                    counts=counts)
+        return {"points": {nm: fake_point(nm) for nm in points}, "headline": headline,
+                "clocks": {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}}
 
     monkeypatch.setattr(bench, "run_cuda", fake_run)
     monkeypatch.setattr(sys, "argv", ["bench.py", "--steps", "20", "--warmup", "3", "--no-cpu-baseline"])
@@ -126,7 +134,30 @@ def test_bench_line_has_the_contract_keys(monkeypatch, capsys):
     for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
                 "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "clocks", "gpu_launches"):
         assert key in line, key
-    assert line["config"]["workload"] == bench.DEFAULT_WORKLOAD
-    assert line["roofline"]["bound"] == "hbm" and 0 < line["roofline"]["frac"]
-    assert line["e2e"]["value"] > 0 and line["gpu_launches"] == 140
-    assert line["value"] == pytest.approx(flops / 0.08e-3 / 1e12)
+    assert line["config"]["workload"] == bench.DEFAULT_WORKLOAD and line["config"]["headline"] == headline
+    assert line["config"]["experts"] == 384 and line["config"]["tokens_per_gpu"] == 4096
+    assert 0 < line["roofline"]["frac"]
+    assert line["e2e"]["value"] > 0 and line["gpu_launches"] == 20 * (4 + 2 + 3)
+    flops = fake_point(headline)["flops"]
+    assert line["value"] == pytest.approx(flops / 0.5e-3 / 1e12)
+    assert [e["workload"] for e in line["sweep"]] == points
+    assert {e["tokens"] for e in line["sweep"]} == set(bench.LAYER_T)
+    assert all(set(e["gemms"]) == {"gate_up", "down"} for e in line["sweep"])
+
+
+def test_gpus_flag_must_match_the_launcher(monkeypatch):
+    """Under a launcher, --gpus must equal WORLD_SIZE."""
+    import sys
+    import bench
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--gpus", "4"])
+    with pytest.raises(SystemExit):
+        bench.main()
+
+
+def test_fixed_count_logits_give_the_asked_counts():
+    import bench
+    import oracle as O
+    want = [4, 0, 2, 6, 4]
+    rt = O.route(bench.fixed_count_logits(8, want, k=2), 2)
+    assert list(rt.counts) == want
