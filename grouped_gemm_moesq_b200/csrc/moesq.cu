@@ -14,6 +14,7 @@
 #include "../../include/moesq.h"
 #include "common.cuh"
 #include "gemm.cuh"
+#include "gemm_pair.cuh"
 #include "pack.cuh"
 #include "peak.cuh"
 #include "quant.cuh"
@@ -79,7 +80,8 @@ moesq_status launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sm
 
 struct DeviceInfo {
   int sms = 0;
-  bool gemm_attr64 = false, gemm_attr128 = false;
+  bool gemm_attr64 = false, gemm_attr128 = false, gemm_attr_pair = false;
+  int pair_clusters = 0;     // co-resident clusters of the SM-pair GEMM
 };
 
 DeviceInfo& device_info() {
@@ -178,6 +180,66 @@ moesq_status launch_gemm(const moesq_weights* w, const uint8_t* a_codes, const u
   p.timeout_ns = g_timeout_ns;
   const int grid = num_ctas > 0 ? num_ctas : di.sms * C::kCtasPerSm;
   return launch_pdl(grouped_sparse_gemm_kernel<TN>, dim3(grid), dim3(kGemmThreads), (size_t)C::kSmemBytes, s, tmb, p);
+}
+
+// SM-pair GEMM (cta_group::2): 256-row weight tiles, 128-row token tiles.
+moesq_status launch_gemm_pair(const moesq_weights* w, const uint8_t* a_codes, const uint8_t* a_scales, int rows_cap,
+                              const int32_t* counts, const int32_t* row_offsets, const float* gamma_a, uint16_t* y,
+                              int num_ctas, cudaStream_t s) {
+  using C = PairCfg;
+  DeviceInfo& di = device_info();
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  if (!di.gemm_attr_pair) {
+    MOESQ_CUDA(cudaFuncSetAttribute(grouped_sparse_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    C::kSmemBytes));
+    cfg.gridDim = dim3(2 * di.sms);
+    int ncl = 0;
+    MOESQ_CUDA(cudaOccupancyMaxActiveClusters(&ncl, grouped_sparse_gemm_pair_kernel, &cfg));
+    if (ncl < 1) return MOESQ_ERR_UNSUPPORTED_SHAPE;
+    di.pair_clusters = ncl;
+    di.gemm_attr_pair = true;
+  }
+  const int64_t KT = w->K / 256;
+  PairMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  if (!make_tmap(&maps.tok, a_codes, (uint64_t)w->K / 2, (uint64_t)rows_cap, 128, 32, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap(&maps.wt, w->ktiles, 128, (uint64_t)w->E * (w->M / 128) * KT * (kKTileBytes / 128), 128,
+                 kKTileBytes / 128, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tmap(&maps.sf, a_scales, 256, (uint64_t)(rows_cap / 128) * (w->K / 128) * 2, 256, 4,
+                 CU_TENSOR_MAP_SWIZZLE_NONE))
+    return MOESQ_ERR_CUDA;
+  GemmParams p;
+  p.ktiles = w->ktiles;
+  p.a_scales = a_scales;
+  p.gamma_w = w->global_scale;
+  p.gamma_a = gamma_a;
+  p.counts = counts;
+  p.row_offsets = row_offsets;
+  p.y = y;
+  p.E = w->E;
+  p.M = w->M;
+  p.K = w->K;
+  p.rows_cap = rows_cap;
+  p.timeout_ns = g_timeout_ns;
+  int ncl = di.pair_clusters;
+  if (num_ctas > 0) ncl = std::max(1, std::min(ncl, num_ctas / 2));
+  cfg.gridDim = dim3(2 * ncl);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, grouped_sparse_gemm_pair_kernel, maps, p);
+  if (e == cudaSuccess) return MOESQ_OK;
+  t_last_cuda_error = e;
+  return MOESQ_ERR_CUDA;
 }
 
 // Layer workspace carve-up.
@@ -501,7 +563,12 @@ moesq_status moesq_grouped_sparse_gemm(const moesq_weights* w, const uint8_t* a_
   const int sm_mode = cfg ? cfg->sm_mode : 0;
   if (tile_n != 0 && tile_n != 64 && tile_n != 128) return MOESQ_ERR_INVALID_ARG;
   if (num_ctas < 0 || sm_mode < 0 || sm_mode > 2) return MOESQ_ERR_INVALID_ARG;
-  if (sm_mode == 2) return MOESQ_ERR_UNSUPPORTED_SHAPE;
+  if (sm_mode == 2) {
+    if (w->M % 256 || (tile_n != 0 && tile_n != 128)) return MOESQ_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned(a_scales, 16)) return MOESQ_ERR_INVALID_ARG;
+    return launch_gemm_pair(w, a_codes, a_scales, rows_cap, counts, row_offsets, gamma_a, y_bf16, num_ctas,
+                            as_stream(stream));
+  }
   if (tile_n == 0) {
     // The counts stay on the device.  The aligned row capacity, less the
     // padding of at most 127 rows per expert, bounds the mean rows per expert.
@@ -521,7 +588,8 @@ moesq_status moesq_gemm_autotune(const moesq_weights* w, const uint8_t* a_codes,
   if (!best || !best_ms || reps < 1) return MOESQ_ERR_INVALID_ARG;
   cudaStream_t s = as_stream(stream);
   const int sms = device_info().sms;
-  const moesq_gemm_config cands[4] = {{64, 2 * sms, 1}, {128, 2 * sms, 1}, {64, sms, 1}, {128, sms, 1}};
+  const moesq_gemm_config cands[5] = {{64, 2 * sms, 1}, {128, 2 * sms, 1}, {64, sms, 1}, {128, sms, 1},
+                                      {128, 2 * sms, 2}};
   cudaEvent_t ev[2];
   MOESQ_CUDA(cudaEventCreate(&ev[0]));
   if (cudaEventCreate(&ev[1]) != cudaSuccess) {
@@ -531,6 +599,7 @@ moesq_status moesq_gemm_autotune(const moesq_weights* w, const uint8_t* a_codes,
   moesq_status st = MOESQ_OK;
   float best_t = -1.0f;
   for (const moesq_gemm_config& c : cands) {
+    if (c.sm_mode == 2 && w->M % 256) continue;        // SM-pair tiles need M % 256 == 0
     st = moesq_grouped_sparse_gemm(w, a_codes, a_scales, rows_cap, counts, row_offsets, gamma_a, y_bf16, &c, s);
     if (st != MOESQ_OK) break;
     if (cudaEventRecord(ev[0], s) != cudaSuccess) { st = MOESQ_ERR_CUDA; break; }

@@ -268,8 +268,12 @@ typedef struct {
   int32_t num_ctas;    /* persistent CTAs: 0 = two per SM (two independent
                           tensor-core issue streams per SM) */
   int32_t sm_mode;     /* 0 = auto; 1 = one SM per 128-row weight tile;
-                          2 = a pair of SMs per 256-row weight tile (not
-                          built: MOESQ_ERR_UNSUPPORTED_SHAPE) */
+                          2 = a pair of SMs (a cluster of two CTAs, one
+                          tcgen05 cta_group::2 MMA per 256-row weight tile,
+                          each SM staging half of the 128-row token tile);
+                          needs M % 256 == 0 and tile_n 0 or 128
+                          (MOESQ_ERR_UNSUPPORTED_SHAPE otherwise); num_ctas
+                          then caps twice the number of clusters */
 } moesq_gemm_config;
 
 moesq_status moesq_grouped_sparse_gemm(const moesq_weights* w, const uint8_t* a_codes,
@@ -279,8 +283,9 @@ moesq_status moesq_grouped_sparse_gemm(const moesq_weights* w, const uint8_t* a_
                                        const moesq_gemm_config* cfg, void* stream);
 
 /* moesq_gemm_autotune: times moesq_grouped_sparse_gemm on these inputs for
- * each candidate configuration (token tile 64 or 128 rows, x one or two
- * persistent CTAs per SM), one warm-up launch and `reps` timed launches each
+ * each candidate configuration (token tile 64 or 128 rows x one or two
+ * persistent CTAs per SM, and the SM-pair variant when M % 256 == 0), one
+ * warm-up launch and `reps` timed launches each
  * (CUDA events on `stream`), and writes the fastest to *best and its mean
  * time in milliseconds to *best_ms (the paper freezes one kernel variant
  * per problem geometry before CUDA-graph capture, App. D.1).  Writes y_bf16

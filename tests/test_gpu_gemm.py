@@ -54,7 +54,7 @@ def test_gemm_tiny_config(cuda_lib, tile_n):
     assert ok, info[:2]
 
 
-@pytest.mark.parametrize("tile_n,mode", [(64, 1), (128, 1)])
+@pytest.mark.parametrize("tile_n,mode", [(64, 1), (128, 1), (128, 2)])
 @pytest.mark.parametrize("counts", [
     [0, 1, 0, 5, 0, 0, 0, 2],              # empty experts, single rows
     [129, 0, 31, 33, 1, 16, 17, 300],      # ragged: several token blocks, partial last blocks
@@ -68,7 +68,7 @@ def test_gemm_edge_counts(cuda_lib, tile_n, mode, counts):
     assert ok, info[:2]
 
 
-@pytest.mark.parametrize("tile_n,mode", [(0, 0), (64, 1), (128, 1)])
+@pytest.mark.parametrize("tile_n,mode", [(0, 0), (64, 1), (128, 1), (128, 2)])
 def test_gemm_multi_k_tiles_and_m_blocks(cuda_lib, tile_n, mode):
     """K = 7168 (28 K steps: every ring wraps several times), M = 1536."""
     E, M, K = 3, 1536, 7168
@@ -78,7 +78,7 @@ def test_gemm_multi_k_tiles_and_m_blocks(cuda_lib, tile_n, mode):
 
 
 @pytest.mark.parametrize("K", [256, 768])
-@pytest.mark.parametrize("tile_n,mode", [(64, 1), (128, 1)])
+@pytest.mark.parametrize("tile_n,mode", [(64, 1), (128, 1), (128, 2)])
 def test_gemm_odd_k_steps(cuda_lib, K, tile_n, mode):
     """K = 256 and 768: one and three 256-wide K steps, fewer than a ring
     holds, and a count that does not divide it."""
