@@ -80,7 +80,7 @@ moesq_status launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sm
 
 struct DeviceInfo {
   int sms = 0;
-  bool gemm_attr64 = false, gemm_attr128 = false, gemm_attr_pair = false;
+  bool gemm_attr64 = false, gemm_attr128 = false, gemm_attr_pair = false, combine_attr = false;
   int pair_clusters = 0;     // co-resident clusters of the SM-pair GEMM
 };
 
@@ -534,7 +534,8 @@ moesq_status moesq_quantize_act(const uint16_t* x_bf16, int T, int K, const moes
     return MOESQ_ERR_INVALID_ARG;
   }
   cudaStream_t s = as_stream(stream);
-  const int64_t tasks = (int64_t)T * k * ((K + 1023) / 1024);
+  const int64_t tasks = (int64_t)T * ((K + 1023) / 1024);
+  if (tasks >= ((int64_t)1 << 31) || (int64_t)T * k >= ((int64_t)1 << 31)) return MOESQ_ERR_UNSUPPORTED_SHAPE;
   return launch_pdl(quantize_act_kernel, dim3(grid_for(tasks, 8, device_info().sms)), dim3(256), 0, s, x_bf16, T, K,
                     k, ids, s2r, E, gamma, rows_cap, codes, scales);
 }
@@ -631,8 +632,7 @@ moesq_status moesq_swiglu_quant(const uint16_t* y_gu, int I, const moesq_routing
   if (I < 256 || I % 256) return MOESQ_ERR_UNSUPPORTED_SHAPE;
   if (!aligned(y_gu, 16) || !aligned(h_codes, 16)) return MOESQ_ERR_INVALID_ARG;
   const int R = rt->T * rt->k;
-  const int64_t tasks = (int64_t)R * ((I + 1023) / 1024);
-  return launch_pdl(swiglu_quant_kernel, dim3(grid_for(tasks, 8, device_info().sms)), dim3(256), 0, as_stream(stream),
+  return launch_pdl(swiglu_quant_kernel, dim3(grid_for(R, 8, device_info().sms)), dim3(256), 0, as_stream(stream),
                     y_gu, I, R, rt->E, rt->topk_ids, rt->slot_to_row, rt->rows_cap, gamma_h, h_codes, h_scales,
                     (unsigned int*)nullptr);
 }
@@ -641,9 +641,17 @@ moesq_status moesq_combine(const uint16_t* y, int H, const moesq_routing* rt, ui
   MOESQ_TRY(check_routing(rt));
   if (!y || !out || H < 8 || H % 8) return MOESQ_ERR_INVALID_ARG;
   if (!aligned(y, 16) || !aligned(out, 16)) return MOESQ_ERR_INVALID_ARG;
-  const int64_t tasks = (int64_t)rt->T * ((H + 255) / 256);
-  return launch_pdl(combine_kernel, dim3(grid_for(tasks, 8, device_info().sms)), dim3(256), 0, as_stream(stream), y,
-                    H, rt->T, rt->k, rt->topk_w, rt->slot_to_row, rt->rows_cap, out);
+  const int64_t nch = (H + kCombineCols - 1) / kCombineCols;
+  const int64_t blocks = (int64_t)rt->T * nch;
+  if (blocks >= ((int64_t)1 << 31)) return MOESQ_ERR_UNSUPPORTED_SHAPE;
+  const size_t smem = (size_t)rt->k * kCombineCols * 2;
+  DeviceInfo& di = device_info();
+  if (!di.combine_attr) {
+    MOESQ_CUDA(cudaFuncSetAttribute(combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 32 * kCombineCols * 2));
+    di.combine_attr = true;
+  }
+  return launch_pdl(combine_kernel, dim3((unsigned)blocks), dim3(kCombineThreads), smem, as_stream(stream), y, H,
+                    rt->T, rt->k, rt->topk_w, rt->slot_to_row, rt->rows_cap, out, g_timeout_ns);
 }
 
 size_t moesq_layer_workspace_bytes(int T, int k, int E, int H, int I) {
@@ -709,7 +717,7 @@ moesq_status moesq_calibrate_layer(const uint16_t* x_bf16, const float* logits, 
                                       gamma_a_gu, ws.y_gu, nullptr, s));
   MOESQ_CUDA(cudaMemsetAsync(gamma_a_dn, 0, sizeof(float) * E, s));
   const int R = T * k;
-  swiglu_quant_kernel<<<grid_for((int64_t)R * ((I + 1023) / 1024), 8, sms), 256, 0, s>>>(
+  swiglu_quant_kernel<<<grid_for(R, 8, sms), 256, 0, s>>>(
       ws.y_gu, I, R, E, rt.topk_ids, rt.slot_to_row, rt.rows_cap, nullptr, nullptr, nullptr,
       reinterpret_cast<unsigned int*>(gamma_a_dn));
   MOESQ_TRY(last_launch());

@@ -35,12 +35,13 @@ __device__ __forceinline__ uint32_t quantize_block32(const float (&v)[32], float
   return code;
 }
 
-// One warp task = (slot, 1024-element chunk of the slot's token): lane l
-// quantises the scale block [1024 c + 32 l, +32) of x[t] with the slot's
-// expert gamma into the slot's row (the fused dispatch + quantisation).
-// Consecutive tasks walk the chunks, then the k slots of a token, so the
-// token's row is re-read from L2.  Plain form (slot_to_row == nullptr): one
-// slot per token, gamma[0], row = t.
+// One warp task = (token t, 1024-element chunk c of x[t]): lane l loads the
+// scale block [1024 c + 32 l, +32) and takes its amax once, then quantises
+// it for each of the token's k slots with the slot's expert gamma into the
+// slot's row (the fused dispatch + quantisation): the block scale code
+// depends on the slot only through gamma.  Indices stay 32-bit (T * k,
+// rows, K and the task count are below 2^31).  Plain form (slot_to_row ==
+// nullptr): one slot, gamma[0], row = t.
 __global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t* __restrict__ x, int T, int K, int k,
                                                            const int32_t* __restrict__ topk_ids,
                                                            const int32_t* __restrict__ slot_to_row, int E,
@@ -49,40 +50,55 @@ __global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t* __res
   pdl_trigger();
   pdl_wait();
   const int lane = threadIdx.x & 31;
-  const int chunks = (K + 1023) / 1024;
   const int nslots = slot_to_row ? k : 1;
-  const int64_t ntasks = (int64_t)T * nslots * chunks;
-  const int64_t wstride = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t task = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); task < ntasks; task += wstride) {
-    const int64_t slot = task / chunks;
-    const int c = (int)(task - slot * chunks);
-    const int64_t t = slot / nslots;
-    int64_t row = t;
-    float g;
-    if (slot_to_row) {
-      const int e = topk_ids[slot];
-      row = slot_to_row[slot];
-      if (e < 0 || e >= E || row < 0 || row >= rows_cap) {
-        if (lane == 0) record_error(kWhereQuant, kErrFault);
-        continue;
+  const int chunks = (K + 1023) >> 10;
+  const int ntasks = T * chunks;
+  const int wstride = gridDim.x * (blockDim.x >> 5);
+  const int KB = K / 128;
+  for (int task = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); task < ntasks; task += wstride) {
+    const int t = task / chunks;
+    const int k0 = (task - t * chunks) * 1024 + lane * 32;
+    // lane j < nslots holds slot j's row and gamma (row -1: invalid slot)
+    int my_row = -1;
+    float my_g = 0.0f;
+    if (lane < nslots) {
+      if (slot_to_row) {
+        const int slot = t * k + lane;
+        const int e = topk_ids[slot], row = slot_to_row[slot];
+        if (e >= 0 && e < E && row >= 0 && row < rows_cap) {
+          my_row = row;
+          my_g = gamma[e];
+        } else if (k0 == lane * 32) {   // reported once per slot (first chunk)
+          record_error(kWhereQuant, kErrFault);
+        }
+      } else {
+        my_row = t;
+        my_g = gamma[0];
       }
-      g = gamma[e];
-    } else {
-      g = gamma[0];
     }
-    const int k0 = c * 1024 + lane * 32;
-    if (k0 >= K) continue;
+    const bool act = k0 < K;
     float v[32];
-    load32_bf16(x + t * K + k0, v);
-    const uint32_t code = quantize_block32(v, g, codes + row * (K / 2) + k0 / 2);
-    scales[mma_scale_offset(row, k0 / 32, K / 128)] = (uint8_t)code;
+    float a = 0.0f;
+    if (act) {
+      load32_bf16(x + (size_t)t * K + k0, v);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) a = fmaxf(a, fabsf(v[i]));
+    }
+    for (int j = 0; j < nslots; ++j) {
+      const int row = __shfl_sync(0xffffffffu, my_row, j);
+      const float g = __shfl_sync(0xffffffffu, my_g, j);
+      if (row < 0 || !act) continue;
+      const uint32_t code = block_scale_code(g, a);
+      *reinterpret_cast<uint4*>(codes + (size_t)row * (K / 2) + k0 / 2) = quant32(v, block_step(code, g), code == 0);
+      scales[mma_scale_offset(row, k0 / 32, KB)] = (uint8_t)code;
+    }
   }
 }
 
-// SwiGLU + requantisation: one warp task = (slot, 1024 outputs), lane l the
-// scale block [1024 c + 32 l, +32) of h; the slot's expert and row come from
-// the routing arrays.  With amax_bits set (calibration) the per-expert amax
-// of h is accumulated instead.
+// SwiGLU + requantisation: one warp per routed slot; per 1024-element chunk
+// of h, lane l the scale block [1024 c + 32 l, +32); the slot's expert and
+// row come from the routing arrays.  With amax_bits set (calibration) the
+// per-expert amax of h is accumulated instead.
 __global__ void __launch_bounds__(256) swiglu_quant_kernel(const uint16_t* __restrict__ y_gu, int I, int R, int E,
                                                            const int32_t* __restrict__ topk_ids,
                                                            const int32_t* __restrict__ slot_to_row, int rows_cap,
@@ -92,25 +108,23 @@ __global__ void __launch_bounds__(256) swiglu_quant_kernel(const uint16_t* __res
   pdl_trigger();
   pdl_wait();
   const int lane = threadIdx.x & 31;
-  const int chunks = (I + 1023) / 1024;
-  const int64_t ntasks = (int64_t)R * chunks;
-  const int64_t wstride = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t task = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); task < ntasks; task += wstride) {
-    const int64_t slot = task / chunks;
-    const int c = (int)(task - slot * chunks);
+  const int wstride = gridDim.x * (blockDim.x >> 5);
+  for (int slot = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); slot < R; slot += wstride) {
     const int e = topk_ids[slot];
-    const int64_t row = slot_to_row[slot];
+    const int row = slot_to_row[slot];
     if (e < 0 || e >= E || row < 0 || row >= rows_cap) {
       if (lane == 0) record_error(kWhereSwiglu, kErrFault);
       continue;
     }
-    const int i0 = c * 1024 + lane * 32;
-    const bool active = i0 < I;
-    float h[32];
-    if (active) {
-      float u[32];
-      load32_bf16(y_gu + row * (2 * I) + i0, h);          // gate
-      load32_bf16(y_gu + row * (2 * I) + I + i0, u);      // up
+    const uint16_t* yr = y_gu + (size_t)row * (2 * I);
+    const float g_h = amax_bits ? 0.0f : gamma_h[e];
+    float amax = 0.0f;
+    for (int c0 = 0; c0 < I; c0 += 1024) {
+      const int i0 = c0 + lane * 32;
+      if (i0 >= I) continue;
+      float h[32], u[32];
+      load32_bf16(yr + i0, h);          // gate
+      load32_bf16(yr + I + i0, u);      // up
       // SiLU(g) = g / (1 + e^-g) in binary32 with the hardware exponential
       // and divide (a few ulp; for g < -88 the denominator overflows and
       // the quotient is 0)
@@ -119,82 +133,100 @@ __global__ void __launch_bounds__(256) swiglu_quant_kernel(const uint16_t* __res
         const float sg = __fdividef(h[i], __fadd_rn(1.0f, __expf(-h[i])));
         h[i] = __fmul_rn(sg, u[i]);
       }
-    }
-    if (amax_bits) {             // calibration: per-expert amax of h
-      float a = 0.0f;
-      if (active) {
+      if (amax_bits) {           // calibration: per-expert amax of h
 #pragma unroll
-        for (int i = 0; i < 32; ++i) a = fmaxf(a, fabsf(h[i]));
+        for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(h[i]));
+        continue;
       }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-      if (lane == 0) atomicMax(amax_bits + e, __float_as_uint(a));
-      continue;
+      const uint32_t code = quantize_block32(h, g_h, h_codes + (size_t)row * (I / 2) + i0 / 2);
+      h_scales[mma_scale_offset(row, i0 / 32, I / 128)] = (uint8_t)code;
     }
-    if (!active) continue;
-    const uint32_t code = quantize_block32(h, gamma_h[e], h_codes + row * (I / 2) + i0 / 2);
-    h_scales[mma_scale_offset(row, i0 / 32, I / 128)] = (uint8_t)code;
+    if (amax_bits) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      if (lane == 0) atomicMax(amax_bits + e, __float_as_uint(amax));
+    }
   }
 }
 
-// Router-weighted combine: one warp task = (token, 256 columns).  Lane j < k
-// fetches slot j's row and weight; the rows of up to 8 slots are then loaded
-// together and summed in slot order (fp32, j = 0 .. k-1).
-__global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ y, int H, int T, int k,
-                                                      const float* __restrict__ topk_w,
-                                                      const int32_t* __restrict__ slot_to_row, int rows_cap,
-                                                      uint16_t* __restrict__ out) {
+// Router-weighted combine: one CTA per (token, chunk of up to kCombineCols
+// columns).  One thread bulk-copies the chunk of each of the token's k rows
+// into shared memory, all completing on one mbarrier (the copies keep many
+// bytes in flight per SM without holding registers); then thread i sums
+// columns [8 i, 8 i + 8) over the k rows in slot order (fp32, j = 0 .. k-1,
+// w_j * y_j) and writes them as bf16.  A slot whose row is outside
+// [0, rows_cap) contributes nothing and sets the error word.
+constexpr int kCombineCols = 2048;
+constexpr int kCombineThreads = kCombineCols / 8;
+
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const uint16_t* __restrict__ y, int H, int T, int k,
+                                                                  const float* __restrict__ topk_w,
+                                                                  const int32_t* __restrict__ slot_to_row,
+                                                                  int rows_cap, uint16_t* __restrict__ out,
+                                                                  uint64_t timeout_ns) {
+  extern __shared__ __align__(128) uint8_t comb_smem[];           // [k][kCombineCols] bf16
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int s_row[32];
+  __shared__ float s_w[32];
+  __shared__ int s_abort;
   pdl_trigger();
   pdl_wait();
-  const int lane = threadIdx.x & 31;
-  const int chunks = (H + 255) / 256;
-  const int64_t ntasks = (int64_t)T * chunks;
-  const int64_t wstride = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t task = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); task < ntasks; task += wstride) {
-    const int64_t t = task / chunks;
-    const int h0 = (int)(task % chunks) * 256 + lane * 8;
-    const bool active = h0 < H;
-    int my_row = -1;
-    float my_w = 0.0f;
-    if (lane < k) {
-      my_row = slot_to_row[t * k + lane];
-      my_w = topk_w[t * k + lane];
+  const int nch = (H + kCombineCols - 1) / kCombineCols;
+  const int t = (int)blockIdx.x / nch;
+  const int h0 = ((int)blockIdx.x - t * nch) * kCombineCols;
+  const int cols = min(kCombineCols, H - h0);
+  const uint32_t b = smem_u32(&bar);
+  if (threadIdx.x < k) {
+    int row = slot_to_row[(size_t)t * k + threadIdx.x];
+    if (row < 0 || row >= rows_cap) {
+      record_error(kWhereCombine, kErrFault);
+      row = -1;
     }
+    s_row[threadIdx.x] = row;
+    s_w[threadIdx.x] = topk_w[(size_t)t * k + threadIdx.x];
+  }
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    mbar_init(b, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t bytes = 0;
+    for (int j = 0; j < k; ++j) bytes += s_row[j] >= 0 ? (uint32_t)cols * 2u : 0u;
+    mbar_arrive_expect_tx(b, bytes);
+    const uint64_t pol = policy_evict_first();
+    for (int j = 0; j < k; ++j)
+      if (s_row[j] >= 0)
+        bulk_load(smem_u32(comb_smem + (size_t)j * kCombineCols * 2), y + (size_t)s_row[j] * H + h0,
+                  (uint32_t)cols * 2u, b, pol);
+  }
+  const bool ok = mbar_wait(b, 0, timeout_ns, &s_abort);
+  if (!ok && threadIdx.x == 0) record_error(kWhereCombine, kErrTimeout);
+  const int c = threadIdx.x * 8;
+  if (ok && c < cols) {
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int j0 = 0; j0 < k; j0 += 8) {
-      uint4 raw[8];
-      int rows[8];
-      float ws[8];
+    for (int j = 0; j < k; ++j) {
+      if (s_row[j] < 0) continue;
+      const float wj = s_w[j];
+      const uint4 raw = *reinterpret_cast<const uint4*>(comb_smem + ((size_t)j * kCombineCols + c) * 2);
+      const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-      for (int jj = 0; jj < 8; ++jj) {
-        rows[jj] = __shfl_sync(0xffffffffu, my_row, (j0 + jj) & 31);
-        ws[jj] = __shfl_sync(0xffffffffu, my_w, (j0 + jj) & 31);
-        raw[jj] = make_uint4(0u, 0u, 0u, 0u);
-        if (active && j0 + jj < k && rows[jj] >= 0 && rows[jj] < rows_cap)
-          raw[jj] = __ldg(reinterpret_cast<const uint4*>(y + (int64_t)rows[jj] * H + h0));
-      }
-#pragma unroll
-      for (int jj = 0; jj < 8; ++jj) {
-        if (j0 + jj >= k) break;
-        if (rows[jj] < 0 || rows[jj] >= rows_cap) {
-          if (lane == 0) record_error(kWhereCombine, kErrFault);
-          continue;
-        }
-        const uint32_t wd[4] = {raw[jj].x, raw[jj].y, raw[jj].z, raw[jj].w};
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float v = (i & 1) ? bf16hi(wd[i >> 1]) : bf16lo(wd[i >> 1]);
-          acc[i] = __fadd_rn(acc[i], __fmul_rn(ws[jj], v));
-        }
+      for (int i = 0; i < 8; ++i) {
+        const float v = (i & 1) ? bf16hi(wd[i >> 1]) : bf16lo(wd[i >> 1]);
+        acc[i] = __fadd_rn(acc[i], __fmul_rn(wj, v));
       }
     }
-    if (!active) continue;
     uint4 o;
     o.x = f32_to_bf16_bits(acc[0]) | (f32_to_bf16_bits(acc[1]) << 16);
     o.y = f32_to_bf16_bits(acc[2]) | (f32_to_bf16_bits(acc[3]) << 16);
     o.z = f32_to_bf16_bits(acc[4]) | (f32_to_bf16_bits(acc[5]) << 16);
     o.w = f32_to_bf16_bits(acc[6]) | (f32_to_bf16_bits(acc[7]) << 16);
-    *reinterpret_cast<uint4*>(out + t * H + h0) = o;
+    *reinterpret_cast<uint4*>(out + (size_t)t * H + h0 + c) = o;
+  }
+  if (!ok) {                     // let copies still in flight land before the CTA's memory is reused
+    int zero = 0;
+    mbar_wait(b, 0, timeout_ns, &zero);
   }
 }
 
