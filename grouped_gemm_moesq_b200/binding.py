@@ -42,6 +42,11 @@ class moesq_routing(ctypes.Structure):
                 ("slot_to_row", _vp)]
 
 
+class moesq_dense_weights(ctypes.Structure):
+    _fields_ = [("E", _i32), ("M", _i32), ("K", _i32), ("codes", _vp), ("scales", _vp), ("global_scale", _vp),
+                ("dtiles", _vp)]
+
+
 class moesq_gemm_config(ctypes.Structure):
     _fields_ = [("tile_n", _i32), ("num_ctas", _i32), ("sm_mode", _i32)]
 
@@ -75,6 +80,11 @@ def load():
         "moesq_route_workspace_bytes": (_sz, [_c.c_int, _c.c_int]),
         "moesq_route_permute": (_c.c_int, [_vp, _P(moesq_routing), _vp, _sz, _vp]),
         "moesq_route_permute_noalloc": (_c.c_int, [_vp, _P(moesq_routing), _vp]),
+        "moesq_dense_weights_bytes": (_sz, [_c.c_int, _c.c_int, _c.c_int, _P(_sz)]),
+        "moesq_pack_dense_nvfp4": (_c.c_int, [_vp, _c.c_int, _c.c_int, _P(moesq_dense_weights), _vp]),
+        "moesq_expand_scales16": (_c.c_int, [_vp, _c.c_int, _c.c_int, _vp, _vp]),
+        "moesq_grouped_dense_gemm": (_c.c_int, [_P(moesq_dense_weights), _vp, _vp, _c.c_int, _vp, _vp, _vp, _vp,
+                                                _P(moesq_gemm_config), _vp]),
         "moesq_mma_peak": (_c.c_int, [_c.c_int, _c.c_int, _c.c_int, _c.c_int, _c.c_int, _P(_c.c_double), _vp]),
         "moesq_quantize_act": (_c.c_int, [_vp, _c.c_int, _c.c_int, _P(moesq_routing), _vp, _c.c_int, _vp, _vp,
                                           _vp]),
@@ -138,6 +148,22 @@ class PackedWeights:
     def nbytes(self) -> int:
         return sum(t.numel() * t.element_size() for t in
                    (self.values, self.mask, self.scales, self.global_scale, self.ktiles))
+
+
+class DenseWeights:
+    """Device tensors of one dense NVFP4 expert stack (the dense control:
+    storage form + kernel form) and the moesq_dense_weights struct."""
+
+    def __init__(self, E: int, M: int, K: int, device="cuda"):
+        import torch
+        self.E, self.M, self.K = E, M, K
+        u8 = dict(dtype=torch.uint8, device=device)
+        self.codes = torch.empty(E, M, K // 2, **u8)
+        self.scales = torch.empty(E, M, K // 16, **u8)
+        self.global_scale = torch.empty(E, dtype=torch.float32, device=device)
+        self.dtiles = torch.empty(E * M * K // 32768 * 18432, **u8)   # 18 KB per 128 x 256 tile
+        self.struct = moesq_dense_weights(E, M, K, self.codes.data_ptr(), self.scales.data_ptr(),
+                                          self.global_scale.data_ptr(), self.dtiles.data_ptr())
 
 
 class RoutingBuffers:
@@ -311,3 +337,31 @@ def moesq_mma_peak(sparse: bool, n: int, ctas_per_sm: int = 1, with_copies: bool
                                  ctypes.byref(out), _stream(stream)),
            "moesq_mma_peak")
     return out.value
+
+
+def scales16_buffer(rows_cap: int, K: int, device="cuda"):
+    """Token scales, one per 16 K, in the dense MMA's layout (uint8, flat)."""
+    import torch
+    return torch.empty(rows_cap * K // 16, dtype=torch.uint8, device=device)
+
+
+def moesq_dense_weights_bytes(E: int, M: int, K: int) -> int:
+    return load().moesq_dense_weights_bytes(E, M, K, None)
+
+
+def moesq_pack_dense_nvfp4(w_bf16, e_begin: int, e_count: int, out: DenseWeights, stream=None):
+    _check(load().moesq_pack_dense_nvfp4(_ptr(w_bf16), e_begin, e_count, ctypes.byref(out.struct), _stream(stream)),
+           "moesq_pack_dense_nvfp4")
+
+
+def moesq_expand_scales16(a_scales, rows_cap: int, K: int, a_scales16, stream=None):
+    _check(load().moesq_expand_scales16(_ptr(a_scales), rows_cap, K, _ptr(a_scales16), _stream(stream)),
+           "moesq_expand_scales16")
+
+
+def moesq_grouped_dense_gemm(w: DenseWeights, a_codes, a_scales16, rows_cap: int, counts, row_offsets, gamma_a,
+                             y_bf16, tile_n: int = 0, num_ctas: int = 0, sm_mode: int = 0, stream=None):
+    cfg = moesq_gemm_config(tile_n, num_ctas, sm_mode)
+    _check(load().moesq_grouped_dense_gemm(ctypes.byref(w.struct), _ptr(a_codes), _ptr(a_scales16), rows_cap,
+                                           _ptr(counts), _ptr(row_offsets), _ptr(gamma_a), _ptr(y_bf16),
+                                           ctypes.byref(cfg), _stream(stream)), "moesq_grouped_dense_gemm")

@@ -36,6 +36,7 @@
 #pragma once
 #include <cuda.h>
 #include "common.cuh"
+#include "dense.cuh"
 #include "pack.cuh"
 
 namespace moesq {
@@ -43,17 +44,21 @@ namespace moesq {
 constexpr int kGemmMaxE = 512;
 constexpr int kGemmThreads = 192;   // producer, MMA, 4 epilogue warps
 
-template <int TN>
+// DENSE: the dense NVFP4 control (dense.cuh): per K step an 18 KB weight
+// tile (128 x 128 B of codes, 128-byte swizzle, and per-16 scales), token
+// scales one per 16 K (2 KB), four dense MMAs of K = 64 and eight scale
+// copies; otherwise the same kernel.
+template <int TN, bool DENSE = false>
 struct GemmCfg {
   // Two CTAs share an SM: each issues its tcgen05 copies and MMAs from one
   // thread, and two such independent issue streams keep the tensor pipe
   // busier than one.
   static constexpr int kCtasPerSm = 2;
   static constexpr int kNAcc = (TN == 128) ? 1 : 2;     // accumulator buffers (TN columns each)
-  static constexpr int kStages = (TN == 128) ? 3 : 5;
-  static constexpr int kWBytes = kKTileBytes;    // weight tile: A image, metadata, scales
+  static constexpr int kStages = DENSE ? ((TN == 128) ? 2 : 3) : ((TN == 128) ? 3 : 5);
+  static constexpr int kWBytes = DENSE ? kDTileBytes : kKTileBytes;   // weight tile of one K step
   static constexpr int kBBytes = TN * 128;       // token codes, 256 K
-  static constexpr int kSfBytes = 1024;          // token scales: 2 x (32 x 16 B)
+  static constexpr int kSfBytes = DENSE ? 2048 : 1024;   // token scales: 4 (or 2) x (32 x 16 B)
   static constexpr int kOffW = 0;
   static constexpr int kOffB = kOffW + kStages * kWBytes;
   static constexpr int kOffSfb = kOffB + kStages * kBBytes;
@@ -65,10 +70,11 @@ struct GemmCfg {
   static constexpr int kOffTab = kOffMisc + 16;
   static constexpr int kSmemBytes = kOffTab + (3 * kGemmMaxE + 1) * 4 + 1024;
   static constexpr uint32_t kTmemCols = 256;            // half of an SM's tensor memory
-  // TMEM buffer b (of kTBufs) at column kColBuf + 20 b: metadata 4 columns,
-  // weight scales 8, token scales 8
+  // TMEM buffer b (of kTBufs) at column kColBuf + kBufCols b: sparse:
+  // metadata 4 columns, weight scales 8, token scales 8; dense: weight
+  // scales 16, token scales 16
   static constexpr uint32_t kColBuf = kNAcc * TN;
-  static constexpr uint32_t kBufCols = 20;
+  static constexpr uint32_t kBufCols = DENSE ? 32 : 20;
   static_assert(TN == 64 || TN == 128, "token tile");
   static_assert(kWBytes % 1024 == 0 && kBBytes % 1024 == 0, "1 KB aligned stages");
   static_assert(kCtasPerSm * (kSmemBytes + 1024) <= 228 * 1024, "shared memory of the CTAs of one SM");
@@ -115,15 +121,16 @@ __device__ __forceinline__ Tile decode_tile(int t, int MB, int E, const int* ntp
   return tl;
 }
 
-template <int TN>
-__global__ void __launch_bounds__(kGemmThreads, GemmCfg<TN>::kCtasPerSm)
+template <int TN, bool DENSE>
+__global__ void __launch_bounds__(kGemmThreads, GemmCfg<TN, DENSE>::kCtasPerSm)
 grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const GemmParams p) {
-  using C = GemmCfg<TN>;
+  using C = GemmCfg<TN, DENSE>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int MB = p.M / 128, KT = p.K / 256, KB = p.K / 128, E = p.E;
+  const int KSF = DENSE ? p.K / 64 : KB;   // 512-byte token-scale blocks per 128 token rows
 
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
@@ -215,7 +222,7 @@ grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const GemmP
         const uint32_t bytes = C::kWBytes + C::kSfBytes + nbox * 4096;
         const uint8_t* wt = p.ktiles + ((int64_t)tl.e * MB + tl.mb) * KT * C::kWBytes;
         const uint64_t pol_w = (ntp[tl.e + 1] - ntp[tl.e] > 1) ? pol_keep : pol_stream;
-        const uint8_t* xsc = p.a_scales + (int64_t)(tl.row0 >> 7) * KB * 512;
+        const uint8_t* xsc = p.a_scales + (int64_t)(tl.row0 >> 7) * KSF * 512;
         for (int kt = 0; kt < KT; ++kt) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, p.timeout_ns, abort_flag)) {
             record_error(kWhereGemmProducer, kErrTimeout);
@@ -226,7 +233,7 @@ grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const GemmP
           const uint32_t fb = full_bar(stage);
           mbar_arrive_expect_tx(fb, bytes);
           bulk_load(sbase + C::kOffW + stage * C::kWBytes, wt + (int64_t)kt * C::kWBytes, C::kWBytes, fb, pol_w);
-          bulk_load(sbase + C::kOffSfb + stage * C::kSfBytes, xsc + kt * 1024, 1024, fb, pol_x);
+          bulk_load(sbase + C::kOffSfb + stage * C::kSfBytes, xsc + kt * C::kSfBytes, C::kSfBytes, fb, pol_x);
           for (int i = 0; i < nbox; ++i)
             tma_load_2d(sbase + C::kOffB + stage * C::kBBytes + i * 4096, &tm_b, fb, kt * 128, tl.row0 + 32 * i,
                         pol_x);
@@ -266,7 +273,7 @@ grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const GemmP
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(buf * TN);
-        const uint32_t idesc = idesc_sp_nvf4((uint32_t)tl.nmma);
+        const uint32_t idesc = DENSE ? (idesc_sp_nvf4((uint32_t)tl.nmma) & ~(1u << 2)) : idesc_sp_nvf4((uint32_t)tl.nmma);
         for (int kt = 0; kt < KT; ++kt, ++g) {
           const int tb = (int)(g % C::kTBufs);
           if (!mbar_wait(full_bar(stage), phase, p.timeout_ns, abort_flag)) {
@@ -280,17 +287,33 @@ grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const GemmP
           const uint32_t sb = sbase + C::kOffB + stage * C::kBBytes;
           const uint32_t ssb = sbase + C::kOffSfb + stage * C::kSfBytes;
           const uint32_t tbuf = tmem + C::kColBuf + C::kBufCols * (uint32_t)tb;
-          tc_cp_128x128b(tbuf, smem_desc(sa + kKTileMeta, 16, 128, 0));
-          tc_cp_32x128b_x4(tbuf + 4, smem_desc(sa + kKTileScales, 16, 128, 0));
-          tc_cp_32x128b_x4(tbuf + 8, smem_desc(sa + kKTileScales + 512, 16, 128, 0));
-          tc_cp_32x128b_x4(tbuf + 12, smem_desc(ssb, 16, 128, 0));
-          tc_cp_32x128b_x4(tbuf + 16, smem_desc(ssb + 512, 16, 128, 0));
+          if constexpr (DENSE) {
+            // four 64-wide K chunks: weight scales at tbuf + 4 j, token scales at tbuf + 16 + 4 j
 #pragma unroll
-          for (int kb = 0; kb < 2; ++kb) {
-            const uint64_t adesc = smem_desc(sa + kb * 32, 16, 512, 4);     // 64-byte swizzle
-            const uint64_t bdesc = smem_desc(sb + kb * 64, 16, 1024, 2);    // 128-byte swizzle
-            tc_mma_sp_nvf4(d_tmem, adesc, bdesc, tbuf + 2 * kb, idesc, tbuf + 4 + 4 * kb,
-                           tbuf + 12 + 4 * kb + tl.q, (kt | kb) != 0 ? 1u : 0u);
+            for (int j = 0; j < 4; ++j) {
+              tc_cp_32x128b_x4(tbuf + 4 * j, smem_desc(sa + kDTileScales + 512 * j, 16, 128, 0));
+              tc_cp_32x128b_x4(tbuf + 16 + 4 * j, smem_desc(ssb + 512 * j, 16, 128, 0));
+            }
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb) {
+              const uint64_t adesc = smem_desc(sa + kb * 32, 16, 1024, 2);    // 128-byte swizzle
+              const uint64_t bdesc = smem_desc(sb + kb * 32, 16, 1024, 2);
+              tc_mma_nvf4(d_tmem, adesc, bdesc, idesc, tbuf + 4 * kb, tbuf + 16 + 4 * kb + tl.q,
+                          (kt | kb) != 0 ? 1u : 0u);
+            }
+          } else {
+            tc_cp_128x128b(tbuf, smem_desc(sa + kKTileMeta, 16, 128, 0));
+            tc_cp_32x128b_x4(tbuf + 4, smem_desc(sa + kKTileScales, 16, 128, 0));
+            tc_cp_32x128b_x4(tbuf + 8, smem_desc(sa + kKTileScales + 512, 16, 128, 0));
+            tc_cp_32x128b_x4(tbuf + 12, smem_desc(ssb, 16, 128, 0));
+            tc_cp_32x128b_x4(tbuf + 16, smem_desc(ssb + 512, 16, 128, 0));
+#pragma unroll
+            for (int kb = 0; kb < 2; ++kb) {
+              const uint64_t adesc = smem_desc(sa + kb * 32, 16, 512, 4);     // 64-byte swizzle
+              const uint64_t bdesc = smem_desc(sb + kb * 64, 16, 1024, 2);    // 128-byte swizzle
+              tc_mma_sp_nvf4(d_tmem, adesc, bdesc, tbuf + 2 * kb, idesc, tbuf + 4 + 4 * kb,
+                             tbuf + 12 + 4 * kb + tl.q, (kt | kb) != 0 ? 1u : 0u);
+            }
           }
           any = true;
           tc_commit(empty_bar(stage));

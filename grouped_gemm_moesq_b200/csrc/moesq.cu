@@ -13,6 +13,7 @@
 
 #include "../../include/moesq.h"
 #include "common.cuh"
+#include "dense.cuh"
 #include "gemm.cuh"
 #include "gemm_pair.cuh"
 #include "pack.cuh"
@@ -81,6 +82,7 @@ moesq_status launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sm
 struct DeviceInfo {
   int sms = 0;
   bool gemm_attr64 = false, gemm_attr128 = false, gemm_attr_pair = false, combine_attr = false;
+  bool dense_attr64 = false, dense_attr128 = false;
   int pair_clusters = 0;     // co-resident clusters of the SM-pair GEMM
 };
 
@@ -150,36 +152,60 @@ moesq_status check_routing(const moesq_routing* rt) {
   return MOESQ_OK;
 }
 
-template <int TN>
-moesq_status launch_gemm(const moesq_weights* w, const uint8_t* a_codes, const uint8_t* a_scales, int rows_cap,
-                         const int32_t* counts, const int32_t* row_offsets, const float* gamma_a, uint16_t* y,
-                         int num_ctas, cudaStream_t s) {
-  using C = GemmCfg<TN>;
+// One-SM grouped GEMM: the sparse kernel, or (DENSE) the dense NVFP4
+// control; `tiles` is the weights' kernel form.
+template <int TN, bool DENSE>
+moesq_status launch_gemm_tiles(const uint8_t* tiles, const float* gamma_w, int E, int M, int K,
+                               const uint8_t* a_codes, const uint8_t* a_scales, int rows_cap, const int32_t* counts,
+                               const int32_t* row_offsets, const float* gamma_a, uint16_t* y, int num_ctas,
+                               cudaStream_t s) {
+  using C = GemmCfg<TN, DENSE>;
   DeviceInfo& di = device_info();
-  bool& attr = (TN == 128) ? di.gemm_attr128 : di.gemm_attr64;
+  bool& attr = DENSE ? ((TN == 128) ? di.dense_attr128 : di.dense_attr64)
+                     : ((TN == 128) ? di.gemm_attr128 : di.gemm_attr64);
   if (!attr) {
-    MOESQ_CUDA(cudaFuncSetAttribute(grouped_sparse_gemm_kernel<TN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    C::kSmemBytes));
+    MOESQ_CUDA(cudaFuncSetAttribute(grouped_sparse_gemm_kernel<TN, DENSE>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes));
     attr = true;
   }
   CUtensorMap tmb;
-  if (!make_tmap(&tmb, a_codes, (uint64_t)w->K / 2, (uint64_t)rows_cap, 128, 32, CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!make_tmap(&tmb, a_codes, (uint64_t)K / 2, (uint64_t)rows_cap, 128, 32, CU_TENSOR_MAP_SWIZZLE_128B))
     return MOESQ_ERR_CUDA;
   GemmParams p;
-  p.ktiles = w->ktiles;
+  p.ktiles = tiles;
   p.a_scales = a_scales;
-  p.gamma_w = w->global_scale;
+  p.gamma_w = gamma_w;
   p.gamma_a = gamma_a;
   p.counts = counts;
   p.row_offsets = row_offsets;
   p.y = y;
-  p.E = w->E;
-  p.M = w->M;
-  p.K = w->K;
+  p.E = E;
+  p.M = M;
+  p.K = K;
   p.rows_cap = rows_cap;
   p.timeout_ns = g_timeout_ns;
   const int grid = num_ctas > 0 ? num_ctas : di.sms * C::kCtasPerSm;
-  return launch_pdl(grouped_sparse_gemm_kernel<TN>, dim3(grid), dim3(kGemmThreads), (size_t)C::kSmemBytes, s, tmb, p);
+  return launch_pdl(grouped_sparse_gemm_kernel<TN, DENSE>, dim3(grid), dim3(kGemmThreads), (size_t)C::kSmemBytes, s,
+                    tmb, p);
+}
+
+template <int TN>
+moesq_status launch_gemm(const moesq_weights* w, const uint8_t* a_codes, const uint8_t* a_scales, int rows_cap,
+                         const int32_t* counts, const int32_t* row_offsets, const float* gamma_a, uint16_t* y,
+                         int num_ctas, cudaStream_t s) {
+  return launch_gemm_tiles<TN, false>(w->ktiles, w->global_scale, w->E, w->M, w->K, a_codes, a_scales, rows_cap,
+                                      counts, row_offsets, gamma_a, y, num_ctas, s);
+}
+
+moesq_status check_dense_weights(const moesq_dense_weights* w) {
+  if (!w) return MOESQ_ERR_INVALID_ARG;
+  if (w->E < 1 || w->E > kGemmMaxE || w->M < 128 || w->K < 256) return MOESQ_ERR_UNSUPPORTED_SHAPE;
+  if (w->M % 128 || w->K % 256) return MOESQ_ERR_UNSUPPORTED_SHAPE;
+  if (!w->codes || !w->scales || !w->global_scale || !w->dtiles) return MOESQ_ERR_INVALID_ARG;
+  if (!aligned(w->codes, 16) || !aligned(w->dtiles, 16) || !aligned(w->global_scale, 4))
+    return MOESQ_ERR_INVALID_ARG;
+  if ((int64_t)w->E * w->M >= (int64_t)1 << 31) return MOESQ_ERR_UNSUPPORTED_SHAPE;
+  return MOESQ_OK;
 }
 
 // SM-pair GEMM (cta_group::2): 256-row weight tiles, 128-row token tiles.
@@ -580,6 +606,74 @@ moesq_status moesq_grouped_sparse_gemm(const moesq_weights* w, const uint8_t* a_
   if (tile_n == 64)
     return launch_gemm<64>(w, a_codes, a_scales, rows_cap, counts, row_offsets, gamma_a, y_bf16, num_ctas, s);
   return launch_gemm<128>(w, a_codes, a_scales, rows_cap, counts, row_offsets, gamma_a, y_bf16, num_ctas, s);
+}
+
+moesq_status moesq_grouped_dense_gemm(const moesq_dense_weights* w, const uint8_t* a_codes,
+                                      const uint8_t* a_scales16, int rows_cap, const int32_t* counts,
+                                      const int32_t* row_offsets, const float* gamma_a, uint16_t* y_bf16,
+                                      const moesq_gemm_config* cfg, void* stream) {
+  MOESQ_TRY(check_dense_weights(w));
+  if (!a_codes || !a_scales16 || !counts || !row_offsets || !gamma_a || !y_bf16) return MOESQ_ERR_INVALID_ARG;
+  if (rows_cap < 128 || rows_cap % 128) return MOESQ_ERR_INVALID_ARG;
+  if (!aligned(a_codes, 16) || !aligned(a_scales16, 16) || !aligned(y_bf16, 2)) return MOESQ_ERR_INVALID_ARG;
+  int tile_n = cfg ? cfg->tile_n : 0;
+  const int num_ctas = cfg ? cfg->num_ctas : 0;
+  const int sm_mode = cfg ? cfg->sm_mode : 0;
+  if (tile_n != 0 && tile_n != 64 && tile_n != 128) return MOESQ_ERR_INVALID_ARG;
+  if (num_ctas < 0 || sm_mode < 0 || sm_mode > 2) return MOESQ_ERR_INVALID_ARG;
+  if (sm_mode == 2) return MOESQ_ERR_UNSUPPORTED_SHAPE;
+  if (tile_n == 0) {
+    const int64_t rows_est = std::max<int64_t>(0, (int64_t)rows_cap - 127 * (int64_t)w->E);
+    tile_n = rows_est / w->E > 64 ? 128 : 64;
+  }
+  cudaStream_t s = as_stream(stream);
+  if (tile_n == 64)
+    return launch_gemm_tiles<64, true>(w->dtiles, w->global_scale, w->E, w->M, w->K, a_codes, a_scales16, rows_cap,
+                                       counts, row_offsets, gamma_a, y_bf16, num_ctas, s);
+  return launch_gemm_tiles<128, true>(w->dtiles, w->global_scale, w->E, w->M, w->K, a_codes, a_scales16, rows_cap,
+                                      counts, row_offsets, gamma_a, y_bf16, num_ctas, s);
+}
+
+size_t moesq_dense_weights_bytes(int E, int M, int K, size_t* per_tensor) {
+  const size_t emk = (size_t)E * M * K;
+  size_t t[4] = {emk / 2, emk / 16, (size_t)E * 4, emk / 32768 * kDTileBytes};   // 18 KB per 128 x 256 tile
+  size_t sum = 0;
+  for (int i = 0; i < 4; ++i) {
+    if (per_tensor) per_tensor[i] = t[i];
+    sum += align256(t[i]);
+  }
+  return sum;
+}
+
+moesq_status moesq_pack_dense_nvfp4(const uint16_t* w_bf16, int e_begin, int e_count, const moesq_dense_weights* out,
+                                    void* stream) {
+  MOESQ_TRY(check_dense_weights(out));
+  if (!w_bf16 || !aligned(w_bf16, 16)) return MOESQ_ERR_INVALID_ARG;
+  if (e_begin < 0 || e_count < 1 || e_begin + e_count > out->E) return MOESQ_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  const int sms = device_info().sms;
+  const int M = out->M, K = out->K;
+  float* gamma = out->global_scale + e_begin;
+  MOESQ_CUDA(cudaMemsetAsync(gamma, 0, sizeof(float) * e_count, s));
+  const int64_t groups_per_expert = (int64_t)M * K / 8;
+  dense_amax_kernel<<<grid_for(groups_per_expert * e_count, 256, sms), 256, 0, s>>>(
+      w_bf16, groups_per_expert * e_count, groups_per_expert, reinterpret_cast<unsigned int*>(gamma));
+  MOESQ_TRY(last_launch());
+  pack_gamma_kernel<<<(e_count + 255) / 256, 256, 0, s>>>(gamma, e_count);
+  MOESQ_TRY(last_launch());
+  DensePackOut po{out->codes, out->scales, out->global_scale, out->dtiles};
+  const int64_t n_groups = (int64_t)e_count * M * (K / 16);
+  dense_pack_kernel<<<grid_for(n_groups, 256, sms), 256, 0, s>>>(w_bf16, e_begin, n_groups, M, K, po);
+  return last_launch();
+}
+
+moesq_status moesq_expand_scales16(const uint8_t* a_scales, int rows_cap, int K, uint8_t* a_scales16, void* stream) {
+  if (!a_scales || !a_scales16 || !aligned(a_scales, 4) || !aligned(a_scales16, 4)) return MOESQ_ERR_INVALID_ARG;
+  if (rows_cap < 128 || rows_cap % 128 || K < 256 || K % 256) return MOESQ_ERR_UNSUPPORTED_SHAPE;
+  const int64_t n_words = (int64_t)rows_cap * (K / 16) / 4;
+  expand_scales16_kernel<<<grid_for(n_words, 256, device_info().sms), 256, 0, as_stream(stream)>>>(a_scales, n_words,
+                                                                                                  K, a_scales16);
+  return last_launch();
 }
 
 moesq_status moesq_gemm_autotune(const moesq_weights* w, const uint8_t* a_codes, const uint8_t* a_scales,

@@ -296,6 +296,58 @@ moesq_status moesq_gemm_autotune(const moesq_weights* w, const uint8_t* a_codes,
                                  const float* gamma_a, uint16_t* y_bf16, int reps,
                                  moesq_gemm_config* best, float* best_ms, void* stream);
 
+/* ------------------------------------------------------- dense NVFP4 control
+ * The dense NVFP4 grouped GEMM the paper measures its sparse kernel against
+ * (App. D.2: "Dense (transposed)", the same kernel orientation, differing
+ * only in sparsity; Tables 8 and 9, Fig. 1a).  Every weight is kept:
+ * one UE4M3 scale per 16 K elements (the NVFP4 group), Eq. 5's gamma over
+ * the whole expert linear, value codes by Eq. 3 -- 4.5 bits per weight
+ * against the sparse form's 2.75 (Eq. 7).                                  */
+typedef struct {
+  int32_t E, M, K;       /* E <= 512, M % 128 == 0, K % 256 == 0 */
+  uint8_t* codes;        /* [E][M][K/2] E2M1, element 2i in the low nibble of byte i */
+  uint8_t* scales;       /* [E][M][K/16] UE4M3, row-major */
+  float* global_scale;   /* [E] gamma */
+  uint8_t* dtiles;       /* kernel form [E][M/128][K/256][18432]: per tile 128 rows x 128 B of
+                            codes in the 128-byte swizzle (16-byte chunk c of row r at
+                            chunk c ^ (r & 7)), then the scales of the four 64-wide K
+                            chunks in the MMA scale layout */
+} moesq_dense_weights;
+
+/* Bytes of each dense tensor: per_tensor[0..3] (host, may be NULL) = codes,
+ * scales, global_scale, dtiles; returns the sum (each rounded up to 256). */
+size_t moesq_dense_weights_bytes(int E, int M, int K, size_t* per_tensor);
+
+/* moesq_pack_dense_nvfp4: bf16 expert weights [e_count][M][K] -> the dense
+ * NVFP4 form of experts [e_begin, e_begin + e_count) of `out`:
+ * gamma = 448 / (amax / 6) over all weights of the expert linear,
+ * per 16-element group code = RNE_E4M3(gamma * amax_16 / 6) saturating at
+ * 448, s = UE4M3(code) / gamma, value code = RNE_E2M1(w / s) (binary32, one
+ * rounding per operation; a zero group gets codes 0).  w_bf16 is 16-byte
+ * aligned. */
+moesq_status moesq_pack_dense_nvfp4(const uint16_t* w_bf16, int e_begin, int e_count,
+                                    const moesq_dense_weights* out, void* stream);
+
+/* moesq_expand_scales16: activation scales in the MMA scale layout with one
+ * code per 32 K ([rows_cap/128][K/128][512], as moesq_quantize_act writes
+ * them) -> one code per 16 K in the layout the dense MMA reads
+ * ([rows_cap/128][K/64][512]: 64-wide K chunk j, row 32 a + b, 16-group s
+ * at b * 16 + a * 4 + s); each 32-block's code serves both of its halves,
+ * which leaves every dequantised value unchanged. */
+moesq_status moesq_expand_scales16(const uint8_t* a_scales, int rows_cap, int K, uint8_t* a_scales16,
+                                   void* stream);
+
+/* moesq_grouped_dense_gemm: the result moesq_grouped_sparse_gemm defines,
+ * for dense weights: y[r][m] = bf16_RN(alpha_e * sum_k deq(a[r][k]) *
+ * deq(W_e[m][k])), alpha_e = 1 / (w->global_scale[e] * gamma_a[e]), with
+ * the token scales one per 16 K (moesq_expand_scales16).  Same row space,
+ * validation and cfg as the sparse GEMM; sm_mode 2 is not offered
+ * (MOESQ_ERR_UNSUPPORTED_SHAPE). */
+moesq_status moesq_grouped_dense_gemm(const moesq_dense_weights* w, const uint8_t* a_codes,
+                                      const uint8_t* a_scales16, int rows_cap, const int32_t* counts,
+                                      const int32_t* row_offsets, const float* gamma_a, uint16_t* y_bf16,
+                                      const moesq_gemm_config* cfg, void* stream);
+
 /* ------------------------------------------------------------- layer parts
  * moesq_swiglu_quant: h = SiLU(g) * u for every valid row of the gate_up
  * output y_gu [rows_cap][2I] bf16 (g = columns [0, I), u = [I, 2I);

@@ -118,3 +118,43 @@ def bf16_ulp(y: np.ndarray) -> np.ndarray:
     a = np.abs(np.asarray(y, np.float64))
     e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
     return np.where(a > 0, 2.0 ** (e - 7), 0.0)
+
+
+# ---------------------------------------------------------------- dense control
+def dense_storage_to_dtiles(codes: np.ndarray, scales16: np.ndarray) -> np.ndarray:
+    """Dense storage form (codes [E, M, K/2], per-16 scales [E, M, K/16]) ->
+    kernel-form tiles (flat uint8): per (e, 128-row block, 256-wide K step)
+    128 rows x 128 B of codes with 16-byte chunk c of row r at c ^ (r & 7),
+    then the scales of the four 64-wide K chunks in the MMA scale layout."""
+    E, M, K2 = codes.shape
+    K = 2 * K2
+    MB, KT = M // 128, K // 256
+    v = codes.reshape(E, MB, 128, KT, 8, 16).transpose(0, 1, 3, 2, 4, 5)     # [E,MB,KT,r,c,16]
+    r = np.arange(128)[:, None]
+    c = np.arange(8)[None, :]
+    img = np.empty_like(v)
+    img[:, :, :, r, c ^ (r & 7), :] = v[:, :, :, r, c, :]
+    sc = np.stack([np.stack([scales_to_mma(scales16[e, mb * 128:(mb + 1) * 128]) for mb in range(MB)])
+                   for e in range(E)]).reshape(E, MB, KT, 2048)
+    out = np.concatenate([img.reshape(E, MB, KT, 16384), sc], axis=-1)
+    return np.ascontiguousarray(out).reshape(-1)
+
+
+def dtiles_to_dense_storage(flat: np.ndarray, E: int, M: int, K: int):
+    MB, KT = M // 128, K // 256
+    t = flat.reshape(E, MB, KT, 18432)
+    img = t[..., :16384].reshape(E, MB, KT, 128, 8, 16)
+    r = np.arange(128)[:, None]
+    c = np.arange(8)[None, :]
+    v = img[:, :, :, r, c ^ (r & 7), :]
+    codes = v.transpose(0, 1, 3, 2, 4, 5).reshape(E, M, K // 2)
+    sc = t[..., 16384:].reshape(E, MB, KT * 2048)
+    scales = np.stack([np.concatenate([mma_to_scales(np.ascontiguousarray(sc[e, mb]), 128, 2 * K)
+                                       for mb in range(MB)]) for e in range(E)])
+    return np.ascontiguousarray(codes), np.ascontiguousarray(scales)
+
+
+def scales32_to_scales16_mma(scales32: np.ndarray) -> np.ndarray:
+    """Row-major per-32 scales [R, K/32] -> per-16 scales (each twice) in the
+    dense MMA layout (flat)."""
+    return scales_to_mma(np.repeat(scales32, 2, axis=1))

@@ -144,3 +144,29 @@ def test_mma_peak_checks(L):
     assert L.moesq_mma_peak(1, 128, 3, 0, 100, ctypes.byref(out), None) == INVALID
     assert L.moesq_mma_peak(1, 128, 1, 0, 0, ctypes.byref(out), None) == INVALID
     assert L.moesq_mma_peak(1, 128, 1, 2, 100, ctypes.byref(out), None) == INVALID   # with_copies is 0 or 1
+
+
+def dense(E=4, M=256, K=512, **kw):
+    f = dict(codes=P, scales=P, global_scale=P, dtiles=P)
+    f.update(kw)
+    return B.moesq_dense_weights(E, M, K, f["codes"], f["scales"], f["global_scale"], f["dtiles"])
+
+
+def test_dense_control_checks(L):
+    d = dense()
+    args = lambda w, cfg=None: L.moesq_grouped_dense_gemm(ctypes.byref(w), ptr(), ptr(), 256, ptr(), ptr(),  # noqa
+                                                          ptr(), ptr(), ctypes.byref(cfg) if cfg else None, None)
+    assert args(dense(M=100)) == SHAPE
+    assert args(dense(K=384)) == SHAPE
+    assert args(dense(codes=0)) == INVALID
+    assert args(dense(dtiles=P + 8)) == INVALID
+    assert args(d, B.moesq_gemm_config(32, 0, 0)) == INVALID
+    assert args(d, B.moesq_gemm_config(128, 0, 2)) == SHAPE                # no SM-pair form of the control
+    assert L.moesq_pack_dense_nvfp4(ptr(4), 0, 4, ctypes.byref(d), None) == INVALID
+    assert L.moesq_pack_dense_nvfp4(ptr(), 3, 2, ctypes.byref(d), None) == INVALID
+    assert L.moesq_expand_scales16(ptr(), 100, 512, ptr(), None) == SHAPE
+    assert L.moesq_expand_scales16(ptr(), 128, 384, ptr(), None) == SHAPE
+    assert L.moesq_expand_scales16(None, 128, 512, ptr(), None) == INVALID
+    sizes = (ctypes.c_size_t * 4)()
+    L.moesq_dense_weights_bytes(2, 256, 512, sizes)
+    assert list(sizes) == [2 * 256 * 256, 2 * 256 * 32, 8, 2 * 2 * 2 * 18432]

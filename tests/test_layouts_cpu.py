@@ -48,3 +48,26 @@ def test_aligned_rows_and_compact_positions():
     assert list(ro) == [0, 0, 128, 256, 512, 640]
     rows = L.compact_to_rows(counts)
     assert rows.size == counts.sum() and rows[0] == 0 and rows[1] == 128 and rows[-1] == 512 + 4
+
+
+def test_dense_tile_layout_round_trip_and_swizzle():
+    """Dense kernel form: storage -> tiles -> storage is the identity, row r's
+    16-byte chunk c sits at chunk c ^ (r & 7), and the per-16 scales of a
+    64-wide K chunk land in the MMA scale layout."""
+    import layouts as L
+    rng = np.random.default_rng(3)
+    E, M, K = 2, 256, 512
+    codes = rng.integers(0, 256, size=(E, M, K // 2), dtype=np.uint8)
+    sc = rng.integers(0, 127, size=(E, M, K // 16), dtype=np.uint8)
+    t = L.dense_storage_to_dtiles(codes, sc)
+    assert t.size == E * (M // 128) * (K // 256) * 18432
+    c2, s2 = L.dtiles_to_dense_storage(t, E, M, K)
+    assert (c2 == codes).all() and (s2 == sc).all()
+    tile = t[:18432]                                  # e 0, row block 0, K step 0
+    r, c = 5, 3
+    assert (tile[r * 128 + (c ^ (r & 7)) * 16:][:16] == codes[0, r, c * 16:(c + 1) * 16]).all()
+    r, j, s = 70, 2, 1                                # row 70 = 32 * 2 + 6, 64-chunk 2, 16-group 1
+    assert tile[16384 + j * 512 + 6 * 16 + 2 * 4 + s] == sc[0, r, 4 * j + s]
+    s32 = rng.integers(0, 127, size=(128, K // 32), dtype=np.uint8)
+    s16 = L.mma_to_scales(L.scales32_to_scales16_mma(s32), 128, 2 * K)
+    assert (s16[:, 0::2] == s32).all() and (s16[:, 1::2] == s32).all()
