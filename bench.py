@@ -92,6 +92,18 @@ SWEEPS = {
 }
 DEFAULT_WORKLOAD = "kimi_layer"
 
+# The paper's kernel sweep (App. D.2, Table 8): (M, K) of each layer, the
+# maximum per-expert token counts N and the expert-group counts G; expert g
+# receives N * {1, 3/4, 1/2, 1/4}[g % 4] rows.  Sparse kernel and dense
+# NVFP4 control, each with its fastest configuration, on the same
+# activations; speedup = t_dense / t_sparse.
+TAB8 = {
+    "kimi_gate_up": (4096, 7168, (32, 64, 128, 256, 512, 1024), (24, 48, 96, 192, 384)),
+    "kimi_down": (7168, 2048, (32, 64, 128, 256, 512, 1024), (24, 48, 96, 192, 384)),
+    "30b_gate_up": (1536, 2048, (16, 32, 64, 128, 256, 512, 1024), (8, 16, 32, 64, 128)),
+    "30b_down": (2048, 768, (16, 32, 64, 128, 256, 512, 1024), (8, 16, 32, 64, 128)),
+}
+
 FP4_OVER_BF16 = 4.0    # nominal dense tensor-core ratio, fp4 : bf16 (9 : 2.25 PFLOP/s)
 SPARSE_FACTOR = 2.0    # a structured-sparse MMA runs the dense-equivalent contraction at twice the rate
 
@@ -548,6 +560,138 @@ def run_cuda(args, rank, world, local_rank):
     return {"points": results, "headline": headline, "clocks": clocks.summary(), "fp4_peak": fp4_peak}
 
 
+# ------------------------------------------------------------------ sparse vs dense sweep (Table 8)
+def tab8_counts(N, G):
+    return np.array([N * (4 - g % 4) // 4 for g in range(G)], np.int64)
+
+
+def run_tab8(args):
+    """Times the sparse kernel and the dense NVFP4 control over Table 8's
+    G x N grid on one GPU; prints one JSON line with every configuration."""
+    import ctypes
+    import torch
+    import grouped_gemm_moesq_b200 as m
+    from grouped_gemm_moesq_b200 import binding as B
+    from grouped_gemm_moesq_b200 import build as cuda_build
+    cuda_build.build()
+    m.load()
+    dev = "cuda"
+    seed = 1234
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+
+    def time_graph(fn, reps):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        ts = []
+        for _ in range(args.warmup):
+            flush.zero_()
+            g.replay()
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        del g
+        return statistics.median(ts)
+
+    clocks = ClockSampler(0)
+    clocks.start()
+    layers = {}
+    entries = []
+    tot_fl, tot_sp = 0.0, 0.0
+    for layer, (M, K, Ns, Gs) in TAB8.items():
+        Emax = max(Gs)
+        linear = 1 if layer.endswith("down") else 0
+        pw = m.PackedWeights(Emax, M, K)
+        dw = m.DenseWeights(Emax, M, K)
+        for e0 in range(0, Emax, 8):
+            n = min(8, Emax - e0)
+            w = torch.stack([S.expert_weights_bf16_torch(seed, linear, e, M, K, dev) for e in range(e0, e0 + n)])
+            m.moesq_pack_weights(w, e0, n, pw)
+            m.moesq_pack_dense_nvfp4(w, e0, n, dw)
+            del w
+        torch.cuda.synchronize()
+        speedups = []
+        for G in Gs:
+            ws = B.moesq_weights(G, M, K, pw.values.data_ptr(), pw.mask.data_ptr(), pw.scales.data_ptr(),
+                                 pw.global_scale.data_ptr(), pw.ktiles.data_ptr())
+            wd = B.moesq_dense_weights(G, M, K, dw.codes.data_ptr(), dw.scales.data_ptr(),
+                                       dw.global_scale.data_ptr(), dw.dtiles.data_ptr())
+            for N in Ns:
+                counts = tab8_counts(N, G)
+                ro = np.concatenate([[0], np.cumsum((counts + 127) // 128 * 128)]).astype(np.int32)
+                rc = int(ro[-1])
+                x = S.activations_bf16_torch(seed + G, rc, K, dev)
+                ga = torch.empty(1, dtype=torch.float32, device=dev)
+                m.moesq_act_global_scale(x, ga)
+                gam = ga.expand(G).contiguous()
+                codes, scales = m.act_buffers(rc, K)
+                m.moesq_quantize_act(x, rc, K, None, ga, rc, codes, scales)
+                s16 = m.scales16_buffer(rc, K)
+                m.moesq_expand_scales16(scales, rc, K, s16)
+                cnt = torch.from_numpy(counts.astype(np.int32)).to(dev)
+                rof = torch.from_numpy(ro).to(dev)
+                y = torch.empty(rc, M, dtype=torch.bfloat16, device=dev)
+                del x
+                cand_s = [(64, 2 * sms, 1), (128, 2 * sms, 1), (64, sms, 1), (128, sms, 1)] + \
+                         ([(128, 2 * sms, 2)] if M % 256 == 0 else [])
+                cand_d = [(64, 2 * sms), (128, 2 * sms), (64, sms), (128, sms)]
+
+                def sparse(c):
+                    cfg = B.moesq_gemm_config(*c)
+                    B._check(B.load().moesq_grouped_sparse_gemm(
+                        ctypes.byref(ws), B._ptr(codes), B._ptr(scales), rc, B._ptr(cnt), B._ptr(rof), B._ptr(gam),
+                        B._ptr(y), ctypes.byref(cfg), B._stream()), "sparse")
+
+                def dense(c):
+                    cfg = B.moesq_gemm_config(c[0], c[1], 1)
+                    B._check(B.load().moesq_grouped_dense_gemm(
+                        ctypes.byref(wd), B._ptr(codes), B._ptr(s16), rc, B._ptr(cnt), B._ptr(rof), B._ptr(gam),
+                        B._ptr(y), ctypes.byref(cfg), B._stream()), "dense")
+
+                ts = {c: time_graph(lambda c=c: sparse(c), 3) for c in cand_s}
+                td = {c: time_graph(lambda c=c: dense(c), 3) for c in cand_d}
+                bs, bd = min(ts, key=ts.get), min(td, key=td.get)
+                t_s = time_graph(lambda: sparse(bs), args.steps)
+                t_d = time_graph(lambda: dense(bd), args.steps)
+                fl = 2.0 * M * K * counts.sum()
+                tot_fl += fl
+                tot_sp += t_s
+                speedups.append(t_d / t_s)
+                entries.append({"layer": layer, "M": M, "K": K, "G": G, "N": N, "sparse_ms": t_s, "dense_ms": t_d,
+                                "speedup": t_d / t_s, "sparse_tflops": fl / (t_s * 1e-3) / 1e12,
+                                "dense_tflops": fl / (t_d * 1e-3) / 1e12,
+                                "sparse_config": {"tile_n": bs[0], "num_ctas": bs[1], "sm_mode": bs[2]},
+                                "dense_config": {"tile_n": bd[0], "num_ctas": bd[1]}})
+                del codes, scales, s16, y, cnt, rof
+            st, word = m.moesq_get_device_error()
+            if st != 0:
+                raise RuntimeError("%s: device error word %#x" % (layer, word))
+        layers[layer] = {"geomean_speedup": float(np.exp(np.mean(np.log(speedups)))),
+                         "min_speedup": float(min(speedups)), "max_speedup": float(max(speedups)),
+                         "configs": len(speedups)}
+        del pw, dw
+        torch.cuda.empty_cache()
+    clocks.stop()
+    line = {"metric": METRIC, "value": tot_fl / (tot_sp * 1e-3) / 1e12,
+            "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": tot_sp, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "nvfp4 (e2m1 x ue4m3 products, f32 accumulate, bf16 out)",
+            "data": "synthetic (seeded; Table 8 shapes, per-expert counts N x {1, 3/4, 1/2, 1/4})",
+            "config": {"workload": "tab8_sweep", "timing": "CUDA-graph replay of one GEMM launch, median, L2 "
+                       "flushed (256 MiB write) before every replay; each kernel with its fastest configuration",
+                       "value": "sparse effective TFLOP/s summed over the sweep (total flops / total time)"},
+            "layers": layers, "clocks": clocks.summary(), "sweep_tab8": entries,
+            "gpu_launches": 2 * len(entries) * args.steps}
+    print(json.dumps(line))
+
+
 # ------------------------------------------------------------------ oracle (CPU) arm
 _ORACLE_PREP = {}
 
@@ -700,13 +844,17 @@ def main():
     ap.add_argument("--gpus", type=int, default=None)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(set(WORKLOADS) | set(SWEEPS)))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=sorted(set(WORKLOADS) | set(SWEEPS) | {"tab8_sweep"}))
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
 
     if "WORLD_SIZE" not in os.environ and args.gpus is not None and args.gpus > 1:
         sys.exit(launch_ranks(args.gpus))
+    if args.workload == "tab8_sweep":
+        run_tab8(args)
+        return
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

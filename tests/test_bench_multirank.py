@@ -161,3 +161,12 @@ def test_fixed_count_logits_give_the_asked_counts():
     want = [4, 0, 2, 6, 4]
     rt = O.route(bench.fixed_count_logits(8, want, k=2), 2)
     assert list(rt.counts) == want
+
+
+def test_tab8_pattern_and_shapes():
+    """Table 8's per-expert counts N * {1, 3/4, 1/2, 1/4} and its four layers."""
+    import bench
+    assert bench.tab8_counts(32, 8).tolist() == [32, 24, 16, 8, 32, 24, 16, 8]
+    assert set(bench.TAB8) == {"kimi_gate_up", "kimi_down", "30b_gate_up", "30b_down"}
+    assert bench.TAB8["kimi_down"][:2] == (7168, 2048) and bench.TAB8["30b_down"][:2] == (2048, 768)
+    assert len(bench.TAB8["kimi_gate_up"][2]) * len(bench.TAB8["kimi_gate_up"][3]) == 30
