@@ -52,7 +52,9 @@ METRIC = "paired-4:8 NVFP4 grouped GEMM TFLOP/s + weight GB/s vs roofline, per t
 KIMI = (384, 8, 7168, 2048)        # experts, top-k, hidden, intermediate
 LAYER_T = (1, 16, 64, 256, 1024, 4096, 16384)
 
-# name -> (E, k, H, I, T, routing, kind).  kind: "layer" (the whole path),
+# name -> (E, k, H, I, T, routing, kind).  kind: "layer" (the whole path,
+# SwiGLU + requantisation fused into the gate_up GEMM), "layer_unfused" (the
+# same with SwiGLU + requantisation as a kernel of its own),
 # "gemm" (route + quantise + gate_up GEMM), "gemm_down" (route + quantise +
 # down GEMM), "quant_gemm" (fixed grouping, routed once outside the step:
 # activation quantisation + gate_up GEMM, as the paper's kernel benchmark),
@@ -73,6 +75,8 @@ WORKLOADS = {
 for _t in LAYER_T:
     WORKLOADS["kimi_layer_t%d" % _t] = KIMI + (_t, "uniform", "layer")
     WORKLOADS["kimi_layer_t%d_zipf" % _t] = KIMI + (_t, "zipf", "layer")
+WORKLOADS["kimi_layer_t4096_zipf_unfused"] = KIMI + (4096, "zipf", "layer_unfused")
+WORKLOADS["30b_layer_t256_unfused"] = (128, 8, 2048, 768, 256, "uniform", "layer_unfused")
 # The paper's Table 11 setting (App. D, B200): Kimi gate_up over all 384
 # experts, expert g receiving N * {1, 3/4, 1/2, 1/4}[g % 4] rows, timed as
 # activation quantisation + grouped GEMM (bf16 in, bf16 out); the step is
@@ -262,7 +266,9 @@ def step_work(E, k, H, I, T, counts_gu, kind):
         wbytes = touched * packed_weight_bytes(M, K)
         return flops, wbytes, {"down": wbytes + R * (K // 2 + K // 32) + R * M * 2}, {"down": flops}
     gu_w = touched * packed_weight_bytes(2 * I, H)
-    gu_bytes = gu_w + R * (H // 2 + H // 32) + R * 2 * I * 2
+    # output: the bf16 gate_up rows, or (fused layer) the requantised h rows
+    gu_out = R * (I // 2 + I // 32) if kind == "layer" else R * 2 * I * 2
+    gu_bytes = gu_w + R * (H // 2 + H // 32) + gu_out
     gu_fl = 2.0 * 2 * I * H * R
     if kind in ("gemm", "quant_gemm"):
         return gu_fl, gu_w, {"gate_up": gu_bytes}, {"gate_up": gu_fl}
@@ -277,7 +283,7 @@ def launches_per_step(kind, T):
     finishing kernel for T <= 512 tokens, else top-k, count, scan, scatter;
     then quantise and the GEMM, and for the layer SwiGLU, down GEMM, combine."""
     route = 0 if kind.startswith("quant_gemm") else (2 if T <= 512 else 4)
-    return route + 2 + (3 if kind == "layer" else 0)
+    return route + 2 + {"layer": 2, "layer_unfused": 3}.get(kind, 0)
 
 
 def rank_seed(seed, rank):
@@ -366,10 +372,10 @@ def run_cuda(args, rank, world, local_rank):
     # packed 8 experts at a time; shared by every point with the same shapes
     wcache = {}
 
-    def weights(linear, E, M, K):
-        key = (linear, E, M, K)
+    def weights(linear, E, M, K, layout=0):
+        key = (linear, E, M, K, layout)
         if key not in wcache:
-            pw = m.PackedWeights(E, M, K)
+            pw = m.PackedWeights(E, M, K, layout=layout)
             for e0 in range(0, E, 8):
                 n = min(8, E - e0)
                 w = torch.stack([S.expert_weights_bf16_torch(seed, linear, e, M, K, dev) for e in range(e0, e0 + n)])
@@ -396,8 +402,9 @@ def run_cuda(args, rank, world, local_rank):
         if down_main:
             w_main, w_dn = weights(1, E, H, I), None
         else:
-            w_main = weights(0, E, 2 * I, H)
-            w_dn = weights(1, E, H, I) if kind == "layer" else None
+            # the fused layer reads its gate_up stack in the SwiGLU kernel row order
+            w_main = weights(0, E, 2 * I, H, m.LAYOUT_SWIGLU if kind == "layer" else m.LAYOUT_PLAIN)
+            w_dn = weights(1, E, H, I) if kind.startswith("layer") else None
 
         # this rank's batch (independent replicas: weak scaling, no data-path collective)
         K_in = I if down_main else H
@@ -407,7 +414,7 @@ def run_cuda(args, rank, world, local_rank):
         rb = m.RoutingBuffers(T, E, k)
         ga = torch.empty(E, dtype=torch.float32, device=dev)
         gh = torch.empty(E, dtype=torch.float32, device=dev)
-        if kind == "layer":
+        if kind.startswith("layer"):
             ws = torch.empty(m.moesq_layer_workspace_bytes(T, k, E, H, I), dtype=torch.uint8, device=dev)
             m.moesq_calibrate_layer(x, lg, T, k, w_main, w_dn, ga, gh, ws)
             del ws
@@ -415,8 +422,9 @@ def run_cuda(args, rank, world, local_rank):
             m.moesq_act_global_scale(x, ga[:1])
             ga.fill_(float(ga[:1].item()))
         a_codes, a_scales = m.act_buffers(rb.rows_cap, K_in)
-        y_main = torch.empty(rb.rows_cap, w_main.M, dtype=torch.bfloat16, device=dev)
-        if kind == "layer":
+        # the fused layer never materialises the bf16 gate_up output
+        y_main = None if kind == "layer" else torch.empty(rb.rows_cap, w_main.M, dtype=torch.bfloat16, device=dev)
+        if kind.startswith("layer"):
             h_codes, h_scales = m.act_buffers(rb.rows_cap, I)
             y_dn = torch.empty(rb.rows_cap, H, dtype=torch.bfloat16, device=dev)
             out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
@@ -431,8 +439,12 @@ def run_cuda(args, rank, world, local_rank):
 
         def c_gemm_main():
             tn, nc, cps = tuned["main"]
-            m.moesq_grouped_sparse_gemm(w_main, a_codes, a_scales, rb.rows_cap, rb.counts, rb.row_offsets, ga,
-                                        y_main, tile_n=tn, num_ctas=nc, sm_mode=cps)
+            if kind == "layer":     # gate_up GEMM + SwiGLU + requantisation in one kernel
+                m.moesq_grouped_sparse_gemm_swiglu(w_main, a_codes, a_scales, rb.rows_cap, rb.counts, rb.row_offsets,
+                                                   ga, gh, h_codes, h_scales, tile_n=tn, num_ctas=nc, sm_mode=cps)
+            else:
+                m.moesq_grouped_sparse_gemm(w_main, a_codes, a_scales, rb.rows_cap, rb.counts, rb.row_offsets, ga,
+                                            y_main, tile_n=tn, num_ctas=nc, sm_mode=cps)
 
         if kind.startswith("quant_gemm"):     # fixed grouping: routed once, outside the step
             m.moesq_route_permute(lg, rb)
@@ -440,9 +452,10 @@ def run_cuda(args, rank, world, local_rank):
                      ("gemm_main", c_gemm_main)]
         else:
             comps = [("route_quant", c_route_quant), ("gemm_main", c_gemm_main)]
-        if kind == "layer":
-            comps += [("swiglu_quant", lambda: m.moesq_swiglu_quant(y_main, I, rb, gh, h_codes, h_scales)),
-                      ("gemm_down", lambda: m.moesq_grouped_sparse_gemm(
+        if kind == "layer_unfused":
+            comps += [("swiglu_quant", lambda: m.moesq_swiglu_quant(y_main, I, rb, gh, h_codes, h_scales))]
+        if kind.startswith("layer"):
+            comps += [("gemm_down", lambda: m.moesq_grouped_sparse_gemm(
                           w_dn, h_codes, h_scales, rb.rows_cap, rb.counts, rb.row_offsets, gh, y_dn,
                           tile_n=tuned["down"][0], num_ctas=tuned["down"][1], sm_mode=tuned["down"][2])),
                       ("combine", lambda: m.moesq_combine(y_dn, H, rb, out))]
@@ -458,9 +471,13 @@ def run_cuda(args, rank, world, local_rank):
         st, word = m.moesq_get_device_error()
         if st != 0:
             raise RuntimeError("%s: device error word %#x during warm-up" % (name, word))
-        tuned["main"] = m.moesq_gemm_autotune(w_main, a_codes, a_scales, rb.rows_cap, rb.counts, rb.row_offsets,
-                                              ga, y_main, reps=3)[0]
         if kind == "layer":
+            tuned["main"] = m.moesq_gemm_swiglu_autotune(w_main, a_codes, a_scales, rb.rows_cap, rb.counts,
+                                                         rb.row_offsets, ga, gh, h_codes, h_scales, reps=3)[0]
+        else:
+            tuned["main"] = m.moesq_gemm_autotune(w_main, a_codes, a_scales, rb.rows_cap, rb.counts,
+                                                  rb.row_offsets, ga, y_main, reps=3)[0]
+        if kind.startswith("layer"):
             tuned["down"] = m.moesq_gemm_autotune(w_dn, h_codes, h_scales, rb.rows_cap, rb.counts,
                                                   rb.row_offsets, gh, y_dn, reps=3)[0]
         step_eager()                          # outputs of the tuned configuration
@@ -526,7 +543,7 @@ def run_cuda(args, rank, world, local_rank):
         # e2e through the public host-buffer entry point (layer workloads):
         # pinned host input and logits in, output back, inside the timed region
         e2e = None
-        if kind == "layer":
+        if kind.startswith("layer"):
             wsh = torch.empty(m.moesq_layer_host_workspace_bytes(T, k, E, H, I), dtype=torch.uint8, device=dev)
             xh = x.view(torch.int16).cpu().pin_memory()
             lh = torch.from_numpy(lg_np).pin_memory()
@@ -554,7 +571,7 @@ def run_cuda(args, rank, world, local_rank):
                              flops=flops, wbytes=wbytes, gemm_bytes=gemm_bytes, gemm_fl=gemm_fl, e2e=e2e,
                              tuned=dict(tuned), launches=launches_per_step(kind, T), counts=counts)
         del x, lg, rb, a_codes, a_scales, y_main
-        if kind == "layer":
+        if kind.startswith("layer"):
             del h_codes, h_scales, y_dn, out
         torch.cuda.empty_cache()
     return {"points": results, "headline": headline, "clocks": clocks.summary(), "fp4_peak": fp4_peak}
@@ -744,7 +761,7 @@ def oracle_prepare(workload, n_tokens, seed=1234):
     else:
         prep["pk"] = packed(0, 2 * I, H)
         prep["flops"] = 2.0 * 2 * I * H * n * k
-        if kind == "layer":
+        if kind.startswith("layer"):
             prep["pk_dn"] = packed(1, H, I)
             prep["flops"] = 2.0 * 3 * I * H * n * k
             prep["ga"], prep["gh"] = O.calibrate_layer(x, lg, k, prep["pk"], prep["pk_dn"])
@@ -759,7 +776,7 @@ def run_oracle_sample(workload, n_tokens, seed=1234):
     import oracle as O
     p = oracle_prepare(workload, n_tokens, seed)
     t0 = time.perf_counter()
-    if p["kind"] == "layer":
+    if p["kind"].startswith("layer"):
         O.moe_layer(p["x"], p["lg"], p["k"], p["pk"], p["pk_dn"], p["ga"], p["gh"])
     else:
         rt = O.route(p["lg"], p["k"])
@@ -785,7 +802,7 @@ def oracle_sample_tokens(workload):
     few enough touched experts (about 150 M weights to draw and pack) that
     the preparation stays under a minute or so."""
     E, k, H, I, T, routing, kind = WORKLOADS[workload]
-    per_expert = 3 * I * H if kind == "layer" else H * I if kind in ("gemm_down", "quant_gemm_down") else 2 * I * H
+    per_expert = 3 * I * H if kind.startswith("layer") else H * I if kind in ("gemm_down", "quant_gemm_down") else 2 * I * H
     by_macs = int(2.5e9 // (k * per_expert))
     by_prep = int(150e6 // (k * per_expert))
     return max(1, min(T, by_macs, by_prep))
@@ -827,7 +844,7 @@ def point_entry(name, r, peaks):
            "gemm_config": {g: {"tile_n": tn, "num_ctas": nc, "sm_mode": cps}
                            for g, (tn, nc, cps) in r["tuned"].items() if tn}}
     gemms = {}
-    for gname, part in (("gate_up", "gemm_main"), ("down", "gemm_down" if r["kind"] == "layer" else "gemm_main")):
+    for gname, part in (("gate_up", "gemm_main"), ("down", "gemm_down" if r["kind"].startswith("layer") else "gemm_main")):
         if gname in r["gemm_bytes"] and part in r["parts"]:
             rf = gemm_roofline(r["gemm_bytes"][gname], r["gemm_fl"][gname], r["parts"][part], peaks, None, gname)
             gemms[gname] = {"ms": r["parts"][part], "hbm_frac": rf["hbm_frac"], "tensor_frac": rf["tensor_frac"],

@@ -15,6 +15,10 @@ LIB_PATH = os.path.join(_HERE, "libmoesq.so")
 
 ROW_ALIGN = 128
 
+# Kernel row order of a weight stack (moesq_weights.layout)
+LAYOUT_PLAIN = 0
+LAYOUT_SWIGLU = 1     # gate_up rows interleaved by 64 for the fused SwiGLU epilogue
+
 _c = ctypes
 _vp = ctypes.c_void_p
 _i32 = ctypes.c_int32
@@ -33,7 +37,7 @@ class MoesqError(RuntimeError):
 
 class moesq_weights(ctypes.Structure):
     _fields_ = [("E", _i32), ("M", _i32), ("K", _i32), ("values", _vp), ("mask", _vp), ("scales", _vp),
-                ("global_scale", _vp), ("ktiles", _vp)]
+                ("global_scale", _vp), ("ktiles", _vp), ("layout", _i32)]
 
 
 class moesq_routing(ctypes.Structure):
@@ -91,7 +95,11 @@ def load():
         "moesq_act_global_scale": (_c.c_int, [_vp, _i64, _vp, _vp]),
         "moesq_grouped_sparse_gemm": (_c.c_int, [_P(moesq_weights), _vp, _vp, _c.c_int, _vp, _vp, _vp, _vp,
                                                  _P(moesq_gemm_config), _vp]),
-        "moesq_swiglu_quant": (_c.c_int, [_vp, _c.c_int, _P(moesq_routing), _vp, _vp, _vp, _vp]),
+        "moesq_swiglu_quant": (_c.c_int, [_vp, _c.c_int, _P(moesq_routing), _vp, _vp, _vp, _c.c_int, _vp]),
+        "moesq_grouped_sparse_gemm_swiglu": (_c.c_int, [_P(moesq_weights), _vp, _vp, _c.c_int, _vp, _vp, _vp, _vp,
+                                                        _vp, _vp, _P(moesq_gemm_config), _vp]),
+        "moesq_gemm_swiglu_autotune": (_c.c_int, [_P(moesq_weights), _vp, _vp, _c.c_int, _vp, _vp, _vp, _vp, _vp,
+                                                  _vp, _c.c_int, _P(moesq_gemm_config), _P(_c.c_float), _vp]),
         "moesq_combine": (_c.c_int, [_vp, _c.c_int, _P(moesq_routing), _vp, _vp]),
         "moesq_layer_workspace_bytes": (_sz, [_c.c_int] * 5),
         "moesq_layer_host_workspace_bytes": (_sz, [_c.c_int] * 5),
@@ -131,11 +139,12 @@ def _ptr(t):
 # ------------------------------------------------------------------ buffers
 class PackedWeights:
     """Device tensors of one expert stack (storage form + kernel form) and
-    the moesq_weights struct that points at them."""
+    the moesq_weights struct that points at them.  layout: LAYOUT_PLAIN, or
+    LAYOUT_SWIGLU for a gate_up stack feeding the fused SwiGLU GEMM."""
 
-    def __init__(self, E: int, M: int, K: int, device="cuda"):
+    def __init__(self, E: int, M: int, K: int, device="cuda", layout: int = LAYOUT_PLAIN):
         import torch
-        self.E, self.M, self.K = E, M, K
+        self.E, self.M, self.K, self.layout = E, M, K, layout
         u8 = dict(dtype=torch.uint8, device=device)
         self.values = torch.empty(E, M, K // 4, **u8)
         self.mask = torch.empty(E, M, K // 16, **u8)
@@ -143,7 +152,7 @@ class PackedWeights:
         self.global_scale = torch.empty(E, dtype=torch.float32, device=device)
         self.ktiles = torch.empty(E * M * K // 32 * 11, **u8)
         self.struct = moesq_weights(E, M, K, self.values.data_ptr(), self.mask.data_ptr(), self.scales.data_ptr(),
-                                    self.global_scale.data_ptr(), self.ktiles.data_ptr())
+                                    self.global_scale.data_ptr(), self.ktiles.data_ptr(), layout)
 
     def nbytes(self) -> int:
         return sum(t.numel() * t.element_size() for t in
@@ -292,9 +301,32 @@ def moesq_grouped_sparse_gemm(w: PackedWeights, a_codes, a_scales, rows_cap: int
                                             ctypes.byref(cfg), _stream(stream)), "moesq_grouped_sparse_gemm")
 
 
-def moesq_swiglu_quant(y_gu, I: int, rt: RoutingBuffers, gamma_h, h_codes, h_scales, stream=None):
+def moesq_swiglu_quant(y_gu, I: int, rt: RoutingBuffers, gamma_h, h_codes, h_scales, gu_layout: int = LAYOUT_PLAIN,
+                       stream=None):
     _check(load().moesq_swiglu_quant(_ptr(y_gu), I, ctypes.byref(rt.struct), _ptr(gamma_h), _ptr(h_codes),
-                                     _ptr(h_scales), _stream(stream)), "moesq_swiglu_quant")
+                                     _ptr(h_scales), gu_layout, _stream(stream)), "moesq_swiglu_quant")
+
+
+def moesq_grouped_sparse_gemm_swiglu(w: PackedWeights, a_codes, a_scales, rows_cap: int, counts, row_offsets,
+                                     gamma_a, gamma_h, h_codes, h_scales, tile_n: int = 0, num_ctas: int = 0,
+                                     sm_mode: int = 0, stream=None):
+    cfg = moesq_gemm_config(tile_n, num_ctas, sm_mode)
+    _check(load().moesq_grouped_sparse_gemm_swiglu(ctypes.byref(w.struct), _ptr(a_codes), _ptr(a_scales), rows_cap,
+                                                   _ptr(counts), _ptr(row_offsets), _ptr(gamma_a), _ptr(gamma_h),
+                                                   _ptr(h_codes), _ptr(h_scales), ctypes.byref(cfg),
+                                                   _stream(stream)), "moesq_grouped_sparse_gemm_swiglu")
+
+
+def moesq_gemm_swiglu_autotune(w: PackedWeights, a_codes, a_scales, rows_cap: int, counts, row_offsets, gamma_a,
+                               gamma_h, h_codes, h_scales, reps: int = 5, stream=None):
+    """Fastest (tile_n, num_ctas, sm_mode) of the fused gate_up GEMM and its mean time in ms."""
+    cfg = moesq_gemm_config(0, 0)
+    ms = _c.c_float(0.0)
+    _check(load().moesq_gemm_swiglu_autotune(ctypes.byref(w.struct), _ptr(a_codes), _ptr(a_scales), rows_cap,
+                                             _ptr(counts), _ptr(row_offsets), _ptr(gamma_a), _ptr(gamma_h),
+                                             _ptr(h_codes), _ptr(h_scales), reps, ctypes.byref(cfg),
+                                             ctypes.byref(ms), _stream(stream)), "moesq_gemm_swiglu_autotune")
+    return (cfg.tile_n, cfg.num_ctas, cfg.sm_mode), ms.value
 
 
 def moesq_combine(y, H: int, rt: RoutingBuffers, out, stream=None):

@@ -127,6 +127,15 @@ __device__ __forceinline__ uint32_t quant8_r(const float* v, float s_b, float r,
   return e2m1x8(q);
 }
 
+// SwiGLU of one feature: SiLU(g) * u with SiLU(g) = g / (1 + e^-g) in
+// binary32 with the hardware exponential and divide (a few ulp; for
+// g < -88 the denominator overflows and the quotient is 0).  Every kernel
+// that forms h uses this one function, so fused and unfused paths agree
+// bit for bit.
+__device__ __forceinline__ float silu_mul(float g, float u) {
+  return __fmul_rn(__fdividef(g, __fadd_rn(1.0f, __expf(-g))), u);
+}
+
 // Eight values of one block -> four bytes of codes (x / s_b onto E2M1).
 __device__ __forceinline__ uint32_t quant8(const float (&v)[8], float s_b, bool zero_block) {
   if (zero_block) return 0u;
@@ -146,6 +155,17 @@ __device__ __forceinline__ uint4 quant32(const float (&v)[32], float s_b, bool z
   o.z = quant8_r(v + 16, s_b, r, rfin);
   o.w = quant8_r(v + 24, s_b, r, rfin);
   return o;
+}
+
+// Quantises the 32-element block v with global scale gamma: stores the 16
+// code bytes at dst and returns the block's scale code.
+__device__ __forceinline__ uint32_t quantize_block32(const float (&v)[32], float gamma, uint8_t* dst) {
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) a = fmaxf(a, fabsf(v[i]));
+  const uint32_t code = block_scale_code(gamma, a);
+  *reinterpret_cast<uint4*>(dst) = quant32(v, block_step(code, gamma), code == 0);
+  return code;
 }
 
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -210,6 +230,22 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
       if (globaltimer_ns() - t0 > timeout_ns) return false;
     }
   }
+}
+
+// Named barrier `id` over `nthreads` threads (whole warps), returning
+// whether any participating thread passed v = true.
+__device__ __forceinline__ bool bar_red_or(int id, int nthreads, bool v) {
+  uint32_t r;
+  asm volatile("{\n\t.reg .pred p, q;\n\t"
+               "setp.ne.u32 q, %1, 0;\n\t"
+               "bar.red.or.pred p, %2, %3, q;\n\t"
+               "selp.u32 %0, 1, 0, p;\n\t}"
+               : "=r"(r) : "r"((uint32_t)v), "r"(id), "r"(nthreads) : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ void bar_sync_named(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" :: "r"(id), "r"(nthreads) : "memory");
 }
 
 // ------------------------------------------------------------------ TMA / bulk copies

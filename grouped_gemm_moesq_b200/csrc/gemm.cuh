@@ -48,21 +48,30 @@ constexpr int kGemmThreads = 192;   // producer, MMA, 4 epilogue warps
 // tile (128 x 128 B of codes, 128-byte swizzle, and per-16 scales), token
 // scales one per 16 K (2 KB), four dense MMAs of K = 64 and eight scale
 // copies; otherwise the same kernel.
-template <int TN, bool DENSE = false>
+// SWIGLU: the gate_up GEMM with SwiGLU and the NVFP4 requantisation of h
+// in the epilogue (weights in the gate/up-interleaved kernel row order):
+// y_gu never leaves the SM; the epilogue writes h codes and scales.
+template <int TN, bool DENSE = false, bool SWIGLU = false>
 struct GemmCfg {
   // Two CTAs share an SM: each issues its tcgen05 copies and MMAs from one
   // thread, and two such independent issue streams keep the tensor pipe
   // busier than one.
   static constexpr int kCtasPerSm = 2;
   static constexpr int kNAcc = (TN == 128) ? 1 : 2;     // accumulator buffers (TN columns each)
-  static constexpr int kStages = DENSE ? ((TN == 128) ? 2 : 3) : ((TN == 128) ? 3 : 5);
+  static constexpr int kStages = DENSE ? ((TN == 128) ? 2 : 3) : ((TN == 128) ? 3 : (SWIGLU ? 4 : 5));
   static constexpr int kWBytes = DENSE ? kDTileBytes : kKTileBytes;   // weight tile of one K step
   static constexpr int kBBytes = TN * 128;       // token codes, 256 K
   static constexpr int kSfBytes = DENSE ? 2048 : 1024;   // token scales: 4 (or 2) x (32 x 16 B)
   static constexpr int kOffW = 0;
   static constexpr int kOffB = kOffW + kStages * kWBytes;
   static constexpr int kOffSfb = kOffB + kStages * kBBytes;
-  static constexpr int kOffBar = kOffSfb + kStages * kSfBytes;
+  // SwiGLU transpose buffer: 64 token rows of 128 bf16 (64 gate, then 64 up
+  // features) padded to 272 bytes, so that 16-byte reads of 8 consecutive
+  // rows hit 8 different bank groups
+  static constexpr int kXRow = 272;
+  static constexpr int kXBytes = SWIGLU ? 64 * kXRow : 0;
+  static constexpr int kOffX = kOffSfb + kStages * kSfBytes;
+  static constexpr int kOffBar = kOffX + kXBytes;
   static constexpr int kTBufs = 4;                       // rotating TMEM buffers of metadata + scales
   // full[S], empty[S], acc_full[2], acc_empty[2], drain
   static constexpr int kNumBars = 2 * kStages + 5;
@@ -89,6 +98,9 @@ struct GemmParams {
   const int32_t* counts;
   const int32_t* row_offsets;
   uint16_t* y;
+  uint8_t* h_codes;      // SWIGLU: [rows_cap][M/4]
+  uint8_t* h_scales;     // SWIGLU: MMA scale layout, M/2 columns
+  const float* gamma_h;  // SWIGLU: [E]
   int E, M, K, rows_cap;
   uint64_t timeout_ns;
 };
@@ -121,10 +133,10 @@ __device__ __forceinline__ Tile decode_tile(int t, int MB, int E, const int* ntp
   return tl;
 }
 
-template <int TN, bool DENSE>
-__global__ void __launch_bounds__(kGemmThreads, GemmCfg<TN, DENSE>::kCtasPerSm)
+template <int TN, bool DENSE, bool SWIGLU = false>
+__global__ void __launch_bounds__(kGemmThreads, GemmCfg<TN, DENSE, SWIGLU>::kCtasPerSm)
 grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const GemmParams p) {
-  using C = GemmCfg<TN, DENSE>;
+  using C = GemmCfg<TN, DENSE, SWIGLU>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const uint32_t sbase = smem_u32(smem);
@@ -325,6 +337,100 @@ grouped_sparse_gemm_kernel(const __grid_constant__ CUtensorMap tm_b, const GemmP
         int zero = 0;
         tc_commit(drain_bar);
         mbar_wait(drain_bar, 0, p.timeout_ns, &zero);
+      }
+    }
+  } else if constexpr (SWIGLU) {
+    // Warps 2..5 = TMEM lane quadrants 2, 3, 0, 1.  The tile's 128 weight
+    // rows are gate features 64 mb + [0, 64) (quadrants 0, 1) and the up
+    // rows of the same features (quadrants 2, 3).  The epilogue turns the
+    // accumulator, rounded to bf16 as the unfused GEMM writes y, around in
+    // shared memory 64 token rows at a time (a row: the 64 gate features,
+    // then the 64 up features) and hands TMEM back once the second half is
+    // in registers; thread (token tau, block b) then forms h = SiLU(g) u
+    // for features 64 mb + 32 b + [0, 32) of its token and requantises it
+    // with quantize_block32, the function the SwiGLU kernel uses, while the
+    // MMA runs the next tile.
+    const int quad = warp & 3, fb = quad & 1;
+    const int half_off = (quad >= 2 ? 64 : 0) + fb * 32 + lane;   // feature slot of this lane in a row
+    uint8_t* xbuf = smem + C::kOffX;
+    const int ept = threadIdx.x - 64;               // 0..127
+    const int tau = ept & 63, b = ept >> 6;
+    const int I = p.M >> 1, KBH = I / 128;
+    constexpr int kHalves = TN / 64;
+    int it = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+      const Tile tl = decode_tile<TN>(t, MB, E, ntp, rstart, cnt);
+      const int buf = it % C::kNAcc;
+      const uint32_t aph = (uint32_t)(it / C::kNAcc) & 1u;
+      const bool ok = mbar_wait(accf_bar(buf), aph, p.timeout_ns, abort_flag);
+      if (!ok && lane == 0) { record_error(kWhereGemmEpilogue, kErrTimeout); *abort_flag = 1; }
+      // every epilogue warp reaches this barrier once per tile, so all four
+      // leave together; it also orders the previous tile's reads of the
+      // transpose buffer before this tile's writes
+      if (bar_red_or(1, 128, !ok)) break;
+      tc_fence_after();
+      const float alpha = __frcp_rn(__fmul_rn(p.gamma_w[tl.e], p.gamma_a[tl.e]));
+      const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * TN);
+      const int nch = tl.nmma >> 4;
+      uint32_t hold[4][8];                          // second half (TN = 128): bf16 pairs, columns 64 + 16 c + 2 q, +1
+#pragma unroll
+      for (int c = 0; c < TN / 16; ++c) {
+        if (c >= nch) break;
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(taddr + 16 * c, r);
+        tmem_ld_wait();
+        if (c < 4) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            *reinterpret_cast<uint16_t*>(xbuf + (16 * c + j) * C::kXRow + 2 * half_off) =
+                (uint16_t)f32_to_bf16_bits(__fmul_rn(alpha, __uint_as_float(r[j])));
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            hold[c & 3][q] = f32_to_bf16_bits(__fmul_rn(alpha, __uint_as_float(r[2 * q]))) |
+                             (f32_to_bf16_bits(__fmul_rn(alpha, __uint_as_float(r[2 * q + 1]))) << 16);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acce_bar(buf));    // the accumulator goes back to the MMA warp
+      const float g_h = p.gamma_h[tl.e];
+      const int blk = 2 * tl.mb + b;                  // 32-feature scale block of h
+#pragma unroll
+      for (int hf = 0; hf < kHalves; ++hf) {
+        if (hf == 1) {
+          bar_sync_named(1, 128);                   // the first half has been read
+#pragma unroll
+          for (int c = 4; c < 8; ++c) {
+            if (c >= nch) break;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const uint32_t w2 = hold[c & 3][j >> 1];
+              *reinterpret_cast<uint16_t*>(xbuf + (16 * (c - 4) + j) * C::kXRow + 2 * half_off) =
+                  (uint16_t)((j & 1) ? (w2 >> 16) : (w2 & 0xFFFFu));
+            }
+          }
+        }
+        bar_sync_named(1, 128);                     // this half is in shared memory
+        const int n = 64 * hf + tau;                // token column of this thread
+        if (n < tl.nvalid) {
+          const uint8_t* row = xbuf + tau * C::kXRow;
+          float h[32];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint4 gw = *reinterpret_cast<const uint4*>(row + 64 * b + 16 * k);
+            const uint4 uw = *reinterpret_cast<const uint4*>(row + 128 + 64 * b + 16 * k);
+            const uint32_t g4[4] = {gw.x, gw.y, gw.z, gw.w}, u4[4] = {uw.x, uw.y, uw.z, uw.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              h[8 * k + 2 * q] = silu_mul(bf16lo(g4[q]), bf16lo(u4[q]));
+              h[8 * k + 2 * q + 1] = silu_mul(bf16hi(g4[q]), bf16hi(u4[q]));
+            }
+          }
+          const int64_t row_n = (int64_t)tl.row0 + n;
+          const uint32_t code = quantize_block32(h, g_h, p.h_codes + row_n * (I / 2) + blk * 16);
+          p.h_scales[mma_scale_offset(row_n, blk, KBH)] = (uint8_t)code;
+        }
       }
     }
   } else {

@@ -83,6 +83,7 @@ struct DeviceInfo {
   int sms = 0;
   bool gemm_attr64 = false, gemm_attr128 = false, gemm_attr_pair = false, combine_attr = false;
   bool dense_attr64 = false, dense_attr128 = false;
+  bool swiglu_attr64 = false, swiglu_attr128 = false;
   int pair_clusters = 0;     // co-resident clusters of the SM-pair GEMM
 };
 
@@ -138,6 +139,8 @@ moesq_status check_weights(const moesq_weights* w) {
   if (!aligned(w->values, 16) || !aligned(w->ktiles, 16) || !aligned(w->mask, 2) || !aligned(w->global_scale, 4))
     return MOESQ_ERR_INVALID_ARG;
   if ((int64_t)w->E * w->M >= (int64_t)1 << 31) return MOESQ_ERR_UNSUPPORTED_SHAPE;
+  if (w->layout != MOESQ_LAYOUT_PLAIN && w->layout != MOESQ_LAYOUT_SWIGLU) return MOESQ_ERR_INVALID_ARG;
+  if (w->layout == MOESQ_LAYOUT_SWIGLU && w->M % 256) return MOESQ_ERR_UNSUPPORTED_SHAPE;
   return MOESQ_OK;
 }
 
@@ -152,41 +155,55 @@ moesq_status check_routing(const moesq_routing* rt) {
   return MOESQ_OK;
 }
 
-// One-SM grouped GEMM: the sparse kernel, or (DENSE) the dense NVFP4
-// control; `tiles` is the weights' kernel form.
-template <int TN, bool DENSE>
+// Output of a one-SM GEMM launch: y (bf16), or with SWIGLU the requantised
+// h (codes, scales, gamma_h).
+struct GemmOut {
+  uint16_t* y;
+  uint8_t* h_codes;
+  uint8_t* h_scales;
+  const float* gamma_h;
+};
+
+// One-SM grouped GEMM: the sparse kernel, (DENSE) the dense NVFP4 control,
+// or (SWIGLU) the gate_up GEMM with the SwiGLU requantisation in its
+// epilogue; `tiles` is the weights' kernel form.
+template <int TN, bool DENSE, bool SWIGLU = false>
 moesq_status launch_gemm_tiles(const uint8_t* tiles, const float* gamma_w, int E, int M, int K,
                                const uint8_t* a_codes, const uint8_t* a_scales, int rows_cap, const int32_t* counts,
-                               const int32_t* row_offsets, const float* gamma_a, uint16_t* y, int num_ctas,
+                               const int32_t* row_offsets, const float* gamma_a, const GemmOut& out, int num_ctas,
                                cudaStream_t s) {
-  using C = GemmCfg<TN, DENSE>;
+  using C = GemmCfg<TN, DENSE, SWIGLU>;
   DeviceInfo& di = device_info();
-  bool& attr = DENSE ? ((TN == 128) ? di.dense_attr128 : di.dense_attr64)
-                     : ((TN == 128) ? di.gemm_attr128 : di.gemm_attr64);
+  bool& attr = SWIGLU  ? ((TN == 128) ? di.swiglu_attr128 : di.swiglu_attr64)
+               : DENSE ? ((TN == 128) ? di.dense_attr128 : di.dense_attr64)
+                       : ((TN == 128) ? di.gemm_attr128 : di.gemm_attr64);
   if (!attr) {
-    MOESQ_CUDA(cudaFuncSetAttribute(grouped_sparse_gemm_kernel<TN, DENSE>,
+    MOESQ_CUDA(cudaFuncSetAttribute(grouped_sparse_gemm_kernel<TN, DENSE, SWIGLU>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes));
     attr = true;
   }
   CUtensorMap tmb;
   if (!make_tmap(&tmb, a_codes, (uint64_t)K / 2, (uint64_t)rows_cap, 128, 32, CU_TENSOR_MAP_SWIZZLE_128B))
     return MOESQ_ERR_CUDA;
-  GemmParams p;
+  GemmParams p{};
   p.ktiles = tiles;
   p.a_scales = a_scales;
   p.gamma_w = gamma_w;
   p.gamma_a = gamma_a;
   p.counts = counts;
   p.row_offsets = row_offsets;
-  p.y = y;
+  p.y = out.y;
+  p.h_codes = out.h_codes;
+  p.h_scales = out.h_scales;
+  p.gamma_h = out.gamma_h;
   p.E = E;
   p.M = M;
   p.K = K;
   p.rows_cap = rows_cap;
   p.timeout_ns = g_timeout_ns;
   const int grid = num_ctas > 0 ? num_ctas : di.sms * C::kCtasPerSm;
-  return launch_pdl(grouped_sparse_gemm_kernel<TN, DENSE>, dim3(grid), dim3(kGemmThreads), (size_t)C::kSmemBytes, s,
-                    tmb, p);
+  return launch_pdl(grouped_sparse_gemm_kernel<TN, DENSE, SWIGLU>, dim3(grid), dim3(kGemmThreads),
+                    (size_t)C::kSmemBytes, s, tmb, p);
 }
 
 template <int TN>
@@ -194,7 +211,8 @@ moesq_status launch_gemm(const moesq_weights* w, const uint8_t* a_codes, const u
                          const int32_t* counts, const int32_t* row_offsets, const float* gamma_a, uint16_t* y,
                          int num_ctas, cudaStream_t s) {
   return launch_gemm_tiles<TN, false>(w->ktiles, w->global_scale, w->E, w->M, w->K, a_codes, a_scales, rows_cap,
-                                      counts, row_offsets, gamma_a, y, num_ctas, s);
+                                      counts, row_offsets, gamma_a, GemmOut{y, nullptr, nullptr, nullptr}, num_ctas,
+                                      s);
 }
 
 moesq_status check_dense_weights(const moesq_dense_weights* w) {
@@ -246,7 +264,7 @@ moesq_status launch_gemm_pair(const moesq_weights* w, const uint8_t* a_codes, co
       !make_tmap(&maps.sf, a_scales, 256, (uint64_t)(rows_cap / 128) * (w->K / 128) * 2, 256, 4,
                  CU_TENSOR_MAP_SWIZZLE_NONE))
     return MOESQ_ERR_CUDA;
-  GemmParams p;
+  GemmParams p{};
   p.ktiles = w->ktiles;
   p.a_scales = a_scales;
   p.gamma_w = w->global_scale;
@@ -373,6 +391,7 @@ moesq_status check_layer(int T, int k, const moesq_weights* w_gu, const moesq_we
   if (I2 % 2 || w_dn->K != I2 / 2 || w_dn->M != H) return MOESQ_ERR_INVALID_ARG;
   if (k > std::min(w_gu->E, 32)) return MOESQ_ERR_UNSUPPORTED_SHAPE;
   if ((I2 / 2) % 256) return MOESQ_ERR_UNSUPPORTED_SHAPE;
+  if (w_dn->layout != MOESQ_LAYOUT_PLAIN) return MOESQ_ERR_INVALID_ARG;
   return MOESQ_OK;
 }
 
@@ -383,9 +402,15 @@ moesq_status layer_body(const uint16_t* x, const float* logits, int T, int k, co
   moesq_routing rt = routing_of(ws, T, E, k);
   MOESQ_TRY(moesq_route_permute(logits, &rt, ws.route_ws, moesq_route_workspace_bytes(T, E), s));
   MOESQ_TRY(moesq_quantize_act(x, T, H, &rt, ga_gu, rt.rows_cap, ws.a_codes, ws.a_scales, s));
-  MOESQ_TRY(moesq_grouped_sparse_gemm(w_gu, ws.a_codes, ws.a_scales, rt.rows_cap, rt.counts, rt.row_offsets, ga_gu,
-                                      ws.y_gu, nullptr, s));
-  MOESQ_TRY(moesq_swiglu_quant(ws.y_gu, I, &rt, ga_dn, ws.h_codes, ws.h_scales, s));
+  if (w_gu->layout == MOESQ_LAYOUT_SWIGLU) {
+    // SwiGLU and its requantisation in the gate_up epilogue: y_gu is never written
+    MOESQ_TRY(moesq_grouped_sparse_gemm_swiglu(w_gu, ws.a_codes, ws.a_scales, rt.rows_cap, rt.counts,
+                                               rt.row_offsets, ga_gu, ga_dn, ws.h_codes, ws.h_scales, nullptr, s));
+  } else {
+    MOESQ_TRY(moesq_grouped_sparse_gemm(w_gu, ws.a_codes, ws.a_scales, rt.rows_cap, rt.counts, rt.row_offsets,
+                                        ga_gu, ws.y_gu, nullptr, s));
+    MOESQ_TRY(moesq_swiglu_quant(ws.y_gu, I, &rt, ga_dn, ws.h_codes, ws.h_scales, MOESQ_LAYOUT_PLAIN, s));
+  }
   MOESQ_TRY(moesq_grouped_sparse_gemm(w_dn, ws.h_codes, ws.h_scales, rt.rows_cap, rt.counts, rt.row_offsets, ga_dn,
                                       ws.y_dn, nullptr, s));
   MOESQ_TRY(moesq_combine(ws.y_dn, H, &rt, out, s));
@@ -491,7 +516,7 @@ moesq_status moesq_pack_weights(const uint16_t* w_bf16, int e_begin, int e_count
   MOESQ_TRY(last_launch());
   pack_gamma_kernel<<<(e_count + 255) / 256, 256, 0, s>>>(gamma, e_count);
   MOESQ_TRY(last_launch());
-  PackOut po{out->values, out->mask, out->scales, out->global_scale, out->ktiles};
+  PackOut po{out->values, out->mask, out->scales, out->global_scale, out->ktiles, out->layout};
   const int64_t n_blocks = (int64_t)e_count * M * (K / 32);
   pack_blocks_kernel<<<grid_for(n_blocks, 256, sms), 256, 0, s>>>(w_bf16, e_begin, n_blocks, M, K, po);
   return last_launch();
@@ -504,7 +529,7 @@ moesq_status moesq_import_dense_nvfp4(const uint8_t* codes, const uint8_t* scale
   if (e_begin < 0 || e_count < 1 || e_begin + e_count > out->E) return MOESQ_ERR_INVALID_ARG;
   cudaStream_t s = as_stream(stream);
   const int M = out->M, K = out->K;
-  PackOut po{out->values, out->mask, out->scales, out->global_scale, out->ktiles};
+  PackOut po{out->values, out->mask, out->scales, out->global_scale, out->ktiles, out->layout};
   const int64_t n_blocks = (int64_t)e_count * M * (K / 32);
   import_dense_kernel<<<grid_for(n_blocks, 256, device_info().sms), 256, 0, s>>>(
       codes, scales, global_scale, e_begin, n_blocks, M, K, po, out->global_scale);
@@ -629,9 +654,11 @@ moesq_status moesq_grouped_dense_gemm(const moesq_dense_weights* w, const uint8_
   cudaStream_t s = as_stream(stream);
   if (tile_n == 64)
     return launch_gemm_tiles<64, true>(w->dtiles, w->global_scale, w->E, w->M, w->K, a_codes, a_scales16, rows_cap,
-                                       counts, row_offsets, gamma_a, y_bf16, num_ctas, s);
+                                       counts, row_offsets, gamma_a, GemmOut{y_bf16, nullptr, nullptr, nullptr},
+                                       num_ctas, s);
   return launch_gemm_tiles<128, true>(w->dtiles, w->global_scale, w->E, w->M, w->K, a_codes, a_scales16, rows_cap,
-                                      counts, row_offsets, gamma_a, y_bf16, num_ctas, s);
+                                      counts, row_offsets, gamma_a, GemmOut{y_bf16, nullptr, nullptr, nullptr},
+                                      num_ctas, s);
 }
 
 size_t moesq_dense_weights_bytes(int E, int M, int K, size_t* per_tensor) {
@@ -676,15 +703,16 @@ moesq_status moesq_expand_scales16(const uint8_t* a_scales, int rows_cap, int K,
   return last_launch();
 }
 
-moesq_status moesq_gemm_autotune(const moesq_weights* w, const uint8_t* a_codes, const uint8_t* a_scales,
-                                 int rows_cap, const int32_t* counts, const int32_t* row_offsets,
-                                 const float* gamma_a, uint16_t* y_bf16, int reps,
-                                 moesq_gemm_config* best, float* best_ms, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Times `launch(cfg)` for every candidate (one warm-up launch, then `reps`
+// launches between CUDA events on s) and keeps the fastest.
+template <typename Launch>
+moesq_status autotune_configs(const moesq_gemm_config* cands, int n, int reps, Launch&& launch,
+                              moesq_gemm_config* best, float* best_ms, cudaStream_t s) {
   if (!best || !best_ms || reps < 1) return MOESQ_ERR_INVALID_ARG;
-  cudaStream_t s = as_stream(stream);
-  const int sms = device_info().sms;
-  const moesq_gemm_config cands[5] = {{64, 2 * sms, 1}, {128, 2 * sms, 1}, {64, sms, 1}, {128, sms, 1},
-                                      {128, 2 * sms, 2}};
   cudaEvent_t ev[2];
   MOESQ_CUDA(cudaEventCreate(&ev[0]));
   if (cudaEventCreate(&ev[1]) != cudaSuccess) {
@@ -693,13 +721,12 @@ moesq_status moesq_gemm_autotune(const moesq_weights* w, const uint8_t* a_codes,
   }
   moesq_status st = MOESQ_OK;
   float best_t = -1.0f;
-  for (const moesq_gemm_config& c : cands) {
-    if (c.sm_mode == 2 && w->M % 256) continue;        // SM-pair tiles need M % 256 == 0
-    st = moesq_grouped_sparse_gemm(w, a_codes, a_scales, rows_cap, counts, row_offsets, gamma_a, y_bf16, &c, s);
+  for (int i = 0; i < n && st == MOESQ_OK; ++i) {
+    const moesq_gemm_config& c = cands[i];
+    st = launch(c);
     if (st != MOESQ_OK) break;
     if (cudaEventRecord(ev[0], s) != cudaSuccess) { st = MOESQ_ERR_CUDA; break; }
-    for (int r = 0; r < reps && st == MOESQ_OK; ++r)
-      st = moesq_grouped_sparse_gemm(w, a_codes, a_scales, rows_cap, counts, row_offsets, gamma_a, y_bf16, &c, s);
+    for (int r = 0; r < reps && st == MOESQ_OK; ++r) st = launch(c);
     if (st != MOESQ_OK) break;
     float ms = 0.0f;
     if (cudaEventRecord(ev[1], s) != cudaSuccess || cudaEventSynchronize(ev[1]) != cudaSuccess ||
@@ -719,16 +746,90 @@ moesq_status moesq_gemm_autotune(const moesq_weights* w, const uint8_t* a_codes,
   return st;
 }
 
+}  // namespace
+
+extern "C" {
+
+moesq_status moesq_gemm_autotune(const moesq_weights* w, const uint8_t* a_codes, const uint8_t* a_scales,
+                                 int rows_cap, const int32_t* counts, const int32_t* row_offsets,
+                                 const float* gamma_a, uint16_t* y_bf16, int reps,
+                                 moesq_gemm_config* best, float* best_ms, void* stream) {
+  MOESQ_TRY(check_weights(w));
+  if (!best || !best_ms || reps < 1) return MOESQ_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  const int sms = device_info().sms;
+  const moesq_gemm_config cands[5] = {{64, 2 * sms, 1}, {128, 2 * sms, 1}, {64, sms, 1}, {128, sms, 1},
+                                      {128, 2 * sms, 2}};
+  const int n = (w->M % 256) ? 4 : 5;        // SM-pair tiles need M % 256 == 0
+  return autotune_configs(
+      cands, n, reps,
+      [&](const moesq_gemm_config& c) {
+        return moesq_grouped_sparse_gemm(w, a_codes, a_scales, rows_cap, counts, row_offsets, gamma_a, y_bf16, &c, s);
+      },
+      best, best_ms, s);
+}
+
+moesq_status moesq_grouped_sparse_gemm_swiglu(const moesq_weights* w, const uint8_t* a_codes,
+                                              const uint8_t* a_scales, int rows_cap, const int32_t* counts,
+                                              const int32_t* row_offsets, const float* gamma_a,
+                                              const float* gamma_h, uint8_t* h_codes, uint8_t* h_scales,
+                                              const moesq_gemm_config* cfg, void* stream) {
+  MOESQ_TRY(check_weights(w));
+  if (w->layout != MOESQ_LAYOUT_SWIGLU) return MOESQ_ERR_INVALID_ARG;
+  if (!a_codes || !a_scales || !counts || !row_offsets || !gamma_a || !gamma_h || !h_codes || !h_scales)
+    return MOESQ_ERR_INVALID_ARG;
+  if (rows_cap < 128 || rows_cap % 128) return MOESQ_ERR_INVALID_ARG;
+  if (!aligned(a_codes, 16) || !aligned(a_scales, 16)) return MOESQ_ERR_INVALID_ARG;
+  int tile_n = cfg ? cfg->tile_n : 0;
+  const int num_ctas = cfg ? cfg->num_ctas : 0;
+  const int sm_mode = cfg ? cfg->sm_mode : 0;
+  if (tile_n != 0 && tile_n != 64 && tile_n != 128) return MOESQ_ERR_INVALID_ARG;
+  if (num_ctas < 0 || sm_mode < 0 || sm_mode > 2) return MOESQ_ERR_INVALID_ARG;
+  if (sm_mode == 2) return MOESQ_ERR_UNSUPPORTED_SHAPE;     // one-SM tiles only
+  if (tile_n == 0) {
+    const int64_t rows_est = std::max<int64_t>(0, (int64_t)rows_cap - 127 * (int64_t)w->E);
+    tile_n = rows_est / w->E > 64 ? 128 : 64;
+  }
+  cudaStream_t s = as_stream(stream);
+  const GemmOut out{nullptr, h_codes, h_scales, gamma_h};
+  if (tile_n == 64)
+    return launch_gemm_tiles<64, false, true>(w->ktiles, w->global_scale, w->E, w->M, w->K, a_codes, a_scales,
+                                              rows_cap, counts, row_offsets, gamma_a, out, num_ctas, s);
+  return launch_gemm_tiles<128, false, true>(w->ktiles, w->global_scale, w->E, w->M, w->K, a_codes, a_scales,
+                                             rows_cap, counts, row_offsets, gamma_a, out, num_ctas, s);
+}
+
+moesq_status moesq_gemm_swiglu_autotune(const moesq_weights* w, const uint8_t* a_codes, const uint8_t* a_scales,
+                                        int rows_cap, const int32_t* counts, const int32_t* row_offsets,
+                                        const float* gamma_a, const float* gamma_h, uint8_t* h_codes,
+                                        uint8_t* h_scales, int reps, moesq_gemm_config* best, float* best_ms,
+                                        void* stream) {
+  MOESQ_TRY(check_weights(w));
+  if (w->layout != MOESQ_LAYOUT_SWIGLU) return MOESQ_ERR_INVALID_ARG;
+  if (!best || !best_ms || reps < 1) return MOESQ_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  const int sms = device_info().sms;
+  const moesq_gemm_config cands[4] = {{64, 2 * sms, 1}, {128, 2 * sms, 1}, {64, sms, 1}, {128, sms, 1}};
+  return autotune_configs(
+      cands, 4, reps,
+      [&](const moesq_gemm_config& c) {
+        return moesq_grouped_sparse_gemm_swiglu(w, a_codes, a_scales, rows_cap, counts, row_offsets, gamma_a,
+                                                gamma_h, h_codes, h_scales, &c, s);
+      },
+      best, best_ms, s);
+}
+
 moesq_status moesq_swiglu_quant(const uint16_t* y_gu, int I, const moesq_routing* rt, const float* gamma_h,
-                                uint8_t* h_codes, uint8_t* h_scales, void* stream) {
+                                uint8_t* h_codes, uint8_t* h_scales, int gu_layout, void* stream) {
   MOESQ_TRY(check_routing(rt));
   if (!y_gu || !gamma_h || !h_codes || !h_scales) return MOESQ_ERR_INVALID_ARG;
+  if (gu_layout != MOESQ_LAYOUT_PLAIN && gu_layout != MOESQ_LAYOUT_SWIGLU) return MOESQ_ERR_INVALID_ARG;
   if (I < 256 || I % 256) return MOESQ_ERR_UNSUPPORTED_SHAPE;
   if (!aligned(y_gu, 16) || !aligned(h_codes, 16)) return MOESQ_ERR_INVALID_ARG;
   const int R = rt->T * rt->k;
   return launch_pdl(swiglu_quant_kernel, dim3(grid_for(R, 8, device_info().sms)), dim3(256), 0, as_stream(stream),
                     y_gu, I, R, rt->E, rt->topk_ids, rt->slot_to_row, rt->rows_cap, gamma_h, h_codes, h_scales,
-                    (unsigned int*)nullptr);
+                    (unsigned int*)nullptr, gu_layout);
 }
 
 moesq_status moesq_combine(const uint16_t* y, int H, const moesq_routing* rt, uint16_t* out, void* stream) {
@@ -813,7 +914,7 @@ moesq_status moesq_calibrate_layer(const uint16_t* x_bf16, const float* logits, 
   const int R = T * k;
   swiglu_quant_kernel<<<grid_for(R, 8, sms), 256, 0, s>>>(
       ws.y_gu, I, R, E, rt.topk_ids, rt.slot_to_row, rt.rows_cap, nullptr, nullptr, nullptr,
-      reinterpret_cast<unsigned int*>(gamma_a_dn));
+      reinterpret_cast<unsigned int*>(gamma_a_dn), w_gu->layout);
   MOESQ_TRY(last_launch());
   amax_to_gamma_kernel<<<1, 1024, 0, s>>>(gamma_a_dn, E, 1);
   return last_launch();

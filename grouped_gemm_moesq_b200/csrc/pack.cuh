@@ -78,7 +78,20 @@ struct PackOut {
   uint8_t* scales;    // [E][M][K/32]
   const float* gamma; // [E]
   uint8_t* ktiles;    // [E][M/128][K/256][kKTileBytes]
+  int layout;         // kernel row order: 0 = as stored, 1 = gate/up interleaved by 64 rows
 };
+
+// Kernel-form row of storage row m of an M-row gate_up linear under layout
+// 1: block b of 128 kernel rows holds gate rows [64 b, 64 b + 64) and then
+// up rows M/2 + [64 b, 64 b + 64), so that one 128-row weight tile of the
+// GEMM produces both halves of 64 SwiGLU features.
+__device__ __forceinline__ int kernel_row(int m, int M, int layout) {
+  if (!layout) return m;
+  const int I = M >> 1;
+  const int up = m >= I ? 1 : 0;
+  const int f = m - up * I;
+  return ((f >> 6) << 7) + up * 64 + (f & 63);
+}
 
 // Writes one 32-element block of an expert linear's packed form: the 8 code
 // bytes (the two kept pairs of each of its 4 groups, in K order), the 4 pair
@@ -101,7 +114,8 @@ __device__ __forceinline__ void store_block(const PackOut& out, int e, int m, in
     const uint32_t i1 = 31 - __clz(bits);
     meta |= (i0 | (i1 << 2)) << (4 * g);
   }
-  const int mb = m >> 7, r = m & 127;
+  const int mk_row = kernel_row(m, M, out.layout);
+  const int mb = mk_row >> 7, r = mk_row & 127;
   const int kt = b >> 3, bt = b & 7;            // 32-block within the 256-wide K tile
   uint8_t* tile = out.ktiles + (((int64_t)e * MB + mb) * KT + kt) * kKTileBytes;
   const int chunk = (bt >> 1) ^ ((r >> 1) & 3);  // 16-byte chunk after the swizzle

@@ -24,17 +24,6 @@ __device__ __forceinline__ void load32_bf16(const uint16_t* p, float (&v)[32]) {
   }
 }
 
-// Quantises the 32-element block v with global scale gamma: stores the 16
-// code bytes at dst and returns the block's scale code.
-__device__ __forceinline__ uint32_t quantize_block32(const float (&v)[32], float gamma, uint8_t* dst) {
-  float a = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) a = fmaxf(a, fabsf(v[i]));
-  const uint32_t code = block_scale_code(gamma, a);
-  *reinterpret_cast<uint4*>(dst) = quant32(v, block_step(code, gamma), code == 0);
-  return code;
-}
-
 // One warp task = (token t, 1024-element chunk c of x[t]): lane l loads the
 // scale block [1024 c + 32 l, +32) and takes its amax once, then quantises
 // it for each of the token's k slots with the slot's expert gamma into the
@@ -98,13 +87,16 @@ __global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t* __res
 // SwiGLU + requantisation: one warp per routed slot; per 1024-element chunk
 // of h, lane l the scale block [1024 c + 32 l, +32); the slot's expert and
 // row come from the routing arrays.  With amax_bits set (calibration) the
-// per-expert amax of h is accumulated instead.
+// per-expert amax of h is accumulated instead.  gu_layout gives the column
+// order of y_gu: 0 = [gate 0..I) | up 0..I)], 1 = per 128 columns 64 gate
+// features then the same 64 up features (the kernel row order of weights
+// packed with MOESQ_LAYOUT_SWIGLU).
 __global__ void __launch_bounds__(256) swiglu_quant_kernel(const uint16_t* __restrict__ y_gu, int I, int R, int E,
                                                            const int32_t* __restrict__ topk_ids,
                                                            const int32_t* __restrict__ slot_to_row, int rows_cap,
                                                            const float* __restrict__ gamma_h,
                                                            uint8_t* __restrict__ h_codes, uint8_t* __restrict__ h_scales,
-                                                           unsigned int* __restrict__ amax_bits) {
+                                                           unsigned int* __restrict__ amax_bits, int gu_layout) {
   pdl_trigger();
   pdl_wait();
   const int lane = threadIdx.x & 31;
@@ -123,16 +115,11 @@ __global__ void __launch_bounds__(256) swiglu_quant_kernel(const uint16_t* __res
       const int i0 = c0 + lane * 32;
       if (i0 >= I) continue;
       float h[32], u[32];
-      load32_bf16(yr + i0, h);          // gate
-      load32_bf16(yr + I + i0, u);      // up
-      // SiLU(g) = g / (1 + e^-g) in binary32 with the hardware exponential
-      // and divide (a few ulp; for g < -88 the denominator overflows and
-      // the quotient is 0)
+      const int gcol = gu_layout ? ((i0 >> 6) << 7) + (i0 & 63) : i0;
+      load32_bf16(yr + gcol, h);                        // gate
+      load32_bf16(yr + (gu_layout ? gcol + 64 : I + i0), u);   // up
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float sg = __fdividef(h[i], __fadd_rn(1.0f, __expf(-h[i])));
-        h[i] = __fmul_rn(sg, u[i]);
-      }
+      for (int i = 0; i < 32; ++i) h[i] = silu_mul(h[i], u[i]);
       if (amax_bits) {           // calibration: per-expert amax of h
 #pragma unroll
         for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(h[i]));

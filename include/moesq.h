@@ -103,7 +103,22 @@ void moesq_set_wait_timeout_ns(uint64_t ns);
  *                          each: the scale of row 32a+b and K sub-block s at
  *                          byte b*16 + a*4 + s
  * The kernel form holds the same 11*M*K/32 bytes per expert as the storage
- * form, rearranged so that one K step of the GEMM is one sequential read. */
+ * form, rearranged so that one K step of the GEMM is one sequential read.
+ *
+ * layout orders the rows of the kernel form (the storage form always keeps
+ * the rows as given):
+ *   MOESQ_LAYOUT_PLAIN   kernel row m = storage row m;
+ *   MOESQ_LAYOUT_SWIGLU  for a gate_up linear (M = 2I: gate rows [0, I), up
+ *                        rows [I, 2I)), the 128 kernel rows of block b are
+ *                        gate rows [64 b, 64 b + 64) followed by up rows
+ *                        I + [64 b, 64 b + 64), so that one 128-row weight
+ *                        tile yields both halves of 64 SwiGLU features (the
+ *                        fused SwiGLU + requantisation of App. D.1 "Serving
+ *                        integration"); needs M % 256 == 0.
+ * The grouped GEMM writes its output columns in kernel row order. */
+#define MOESQ_LAYOUT_PLAIN 0
+#define MOESQ_LAYOUT_SWIGLU 1
+
 typedef struct {
   int32_t E, M, K;
   uint8_t* values;
@@ -111,6 +126,7 @@ typedef struct {
   uint8_t* scales;
   float* global_scale;
   uint8_t* ktiles;
+  int32_t layout;      /* MOESQ_LAYOUT_PLAIN or MOESQ_LAYOUT_SWIGLU */
 } moesq_weights;
 
 /* Bytes of each weight tensor: per_tensor[0..4] (host, may be NULL) =
@@ -350,15 +366,48 @@ moesq_status moesq_grouped_dense_gemm(const moesq_dense_weights* w, const uint8_
 
 /* ------------------------------------------------------------- layer parts
  * moesq_swiglu_quant: h = SiLU(g) * u for every valid row of the gate_up
- * output y_gu [rows_cap][2I] bf16 (g = columns [0, I), u = [I, 2I);
- * SiLU(g) = g / (1 + e^-g) in binary32 with the hardware exponential and
- * divide, a few ulp from the exact value), requantised to NVFP4 with
- * gamma_h[e] of the row's expert into h_codes [rows_cap][I/2] and h_scales
- * (MMA scale layout) -- the fused SwiGLU + requantisation of App. D.1.
+ * output y_gu [rows_cap][2I] bf16 (gu_layout MOESQ_LAYOUT_PLAIN: g = columns
+ * [0, I), u = [I, 2I); MOESQ_LAYOUT_SWIGLU: the kernel row order of weights
+ * packed with that layout, feature f at column 128 (f / 64) + f % 64 and its
+ * up half 64 columns later; SiLU(g) = g / (1 + e^-g) in binary32 with the
+ * hardware exponential and divide, a few ulp from the exact value),
+ * requantised to NVFP4 with gamma_h[e] of the row's expert into h_codes
+ * [rows_cap][I/2] and h_scales (MMA scale layout) -- the SwiGLU +
+ * requantisation of App. D.1 as a kernel of its own.
  * I is a multiple of 256; y_gu and h_codes are 16-byte aligned. */
 moesq_status moesq_swiglu_quant(const uint16_t* y_gu, int I, const moesq_routing* rt,
                                 const float* gamma_h, uint8_t* h_codes, uint8_t* h_scales,
-                                void* stream);
+                                int gu_layout, void* stream);
+
+/* moesq_grouped_sparse_gemm_swiglu: the gate_up GEMM with SwiGLU and the
+ * NVFP4 requantisation of h fused into its epilogue (App. D.1 "Serving
+ * integration": "fused SwiGLU with requantization").  w is a gate_up stack
+ * (M = 2I) packed with layout MOESQ_LAYOUT_SWIGLU.  For every valid row r
+ * of expert e the result equals moesq_grouped_sparse_gemm followed by
+ * moesq_swiglu_quant (gu_layout MOESQ_LAYOUT_SWIGLU) bit for bit: g and u
+ * are the bf16-rounded GEMM outputs, h = SiLU(g) * u as there, each 32-wide
+ * block of h gets scale code RNE_E4M3(gamma_h[e] * amax / 6) and the E2M1
+ * codes of the correctly rounded quotients; written to h_codes
+ * [rows_cap][I/2] (row r) and h_scales (MMA scale layout, I / 32 scales per
+ * row).  The bf16 gate_up output never reaches memory.  Same row space,
+ * validation and cfg as moesq_grouped_sparse_gemm, except that sm_mode 2
+ * is not offered (MOESQ_ERR_UNSUPPORTED_SHAPE) and weights of another
+ * layout are rejected (MOESQ_ERR_INVALID_ARG).  a_codes and a_scales are
+ * 16-byte aligned. */
+moesq_status moesq_grouped_sparse_gemm_swiglu(const moesq_weights* w, const uint8_t* a_codes,
+                                              const uint8_t* a_scales, int rows_cap, const int32_t* counts,
+                                              const int32_t* row_offsets, const float* gamma_a,
+                                              const float* gamma_h, uint8_t* h_codes, uint8_t* h_scales,
+                                              const moesq_gemm_config* cfg, void* stream);
+
+/* moesq_gemm_swiglu_autotune: moesq_gemm_autotune for the fused gate_up
+ * GEMM (token tile 64 or 128 rows x one or two CTAs per SM); writes h_codes
+ * and h_scales as the GEMM does; synchronises the stream. */
+moesq_status moesq_gemm_swiglu_autotune(const moesq_weights* w, const uint8_t* a_codes, const uint8_t* a_scales,
+                                        int rows_cap, const int32_t* counts, const int32_t* row_offsets,
+                                        const float* gamma_a, const float* gamma_h, uint8_t* h_codes,
+                                        uint8_t* h_scales, int reps, moesq_gemm_config* best, float* best_ms,
+                                        void* stream);
 
 /* moesq_combine: out[t][h] = bf16( sum_{j<k} topk_w[t][j] * y[slot_to_row[t*k+j]][h] )
  * with binary32 accumulation in slot order (router-weighted token
@@ -371,6 +420,9 @@ moesq_status moesq_combine(const uint16_t* y, int H, const moesq_routing* rt,
  * route + permute -> dispatch-quantise (gamma_a_gu) -> gate_up grouped GEMM
  * (w_gu: M = 2I, K = H) -> SwiGLU + requantise (gamma_a_dn) -> down grouped
  * GEMM (w_dn: M = H, K = I) -> router-weighted combine into out [T][H].
+ * When w_gu has layout MOESQ_LAYOUT_SWIGLU the gate_up GEMM and the SwiGLU
+ * requantisation are one kernel (moesq_grouped_sparse_gemm_swiglu); the
+ * result is the same bit for bit.  w_dn must have layout MOESQ_LAYOUT_PLAIN.
  * x [T][H] bf16, logits [T][E] float32; gamma_a_* [E] float32 (device).
  * All intermediates live in `workspace` (moesq_layer_workspace_bytes).    */
 size_t moesq_layer_workspace_bytes(int T, int k, int E, int H, int I);

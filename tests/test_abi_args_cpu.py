@@ -23,10 +23,10 @@ def L():
     return B.load()
 
 
-def weights(E=4, M=256, K=512, **kw):
+def weights(E=4, M=256, K=512, layout=0, **kw):
     f = dict(values=P, mask=P, scales=P, global_scale=P, ktiles=P)
     f.update(kw)
-    return B.moesq_weights(E, M, K, f["values"], f["mask"], f["scales"], f["global_scale"], f["ktiles"])
+    return B.moesq_weights(E, M, K, f["values"], f["mask"], f["scales"], f["global_scale"], f["ktiles"], layout)
 
 
 def routing(T=8, E=4, k=2, rows_cap=None, **kw):
@@ -104,8 +104,9 @@ def test_quantise_swiglu_combine_checks(L):
     assert L.moesq_quantize_act(ptr(2), 8, 512, ctypes.byref(rt), ptr(), rc, ptr(), ptr(), None) == INVALID
     assert L.moesq_quantize_act(ptr(), 9, 512, ctypes.byref(rt), ptr(), rc, ptr(), ptr(), None) == INVALID
     assert L.moesq_quantize_act(ptr(), 8, 512, None, ptr(), 100, ptr(), ptr(), None) == INVALID
-    assert L.moesq_swiglu_quant(ptr(), 100, ctypes.byref(rt), ptr(), ptr(), ptr(), None) == SHAPE
-    assert L.moesq_swiglu_quant(ptr(), 256, ctypes.byref(rt), ptr(), ptr(8), ptr(), None) == INVALID
+    assert L.moesq_swiglu_quant(ptr(), 100, ctypes.byref(rt), ptr(), ptr(), ptr(), 0, None) == SHAPE
+    assert L.moesq_swiglu_quant(ptr(), 256, ctypes.byref(rt), ptr(), ptr(8), ptr(), 0, None) == INVALID
+    assert L.moesq_swiglu_quant(ptr(), 256, ctypes.byref(rt), ptr(), ptr(), ptr(), 2, None) == INVALID
     assert L.moesq_combine(ptr(), 7, ctypes.byref(rt), ptr(), None) == INVALID
     assert L.moesq_combine(ptr(2), 256, ctypes.byref(rt), ptr(), None) == INVALID
 
@@ -122,6 +123,27 @@ def test_layer_checks(L):
     assert args(ptr(), need, T=0) == INVALID
     assert args(ptr(), need, k=5) == SHAPE                          # top-k above the expert count
     assert args(ptr(), need, wd=weights(E, H, 512)) == INVALID     # down K != I
+    assert args(ptr(), need, wd=weights(E, H, I, layout=1)) == INVALID   # down stack in the SwiGLU order
+
+
+def test_weight_layout_and_fused_gemm_checks(L):
+    def fused(w, cfg=None, h_codes=ptr(), a_scales=ptr()):
+        return L.moesq_grouped_sparse_gemm_swiglu(ctypes.byref(w), ptr(), a_scales, 256, ptr(), ptr(), ptr(), ptr(),
+                                                  h_codes, ptr(), ctypes.byref(cfg) if cfg else None, None)
+    assert gemm(L, weights(layout=2)) == INVALID                    # unknown layout
+    assert gemm(L, weights(M=384, layout=1)) == SHAPE               # SwiGLU order needs M % 256 == 0
+    assert L.moesq_pack_weights(ptr(), 0, 4, ctypes.byref(weights(M=384, layout=1)), None) == SHAPE
+    assert fused(weights()) == INVALID                              # plain order: not a fused gate_up stack
+    assert fused(weights(layout=1), h_codes=None) == INVALID
+    assert fused(weights(layout=1), a_scales=ptr(8)) == INVALID
+    assert fused(weights(layout=1), B.moesq_gemm_config(96, 0, 0)) == INVALID
+    assert fused(weights(layout=1), B.moesq_gemm_config(128, 0, 2)) == SHAPE   # no SM-pair form
+    best, ms = B.moesq_gemm_config(0, 0, 0), ctypes.c_float(0)
+    tune = lambda w, reps: L.moesq_gemm_swiglu_autotune(  # noqa: E731
+        ctypes.byref(w), ptr(), ptr(), 256, ptr(), ptr(), ptr(), ptr(), ptr(), ptr(), reps, ctypes.byref(best),
+        ctypes.byref(ms), None)
+    assert tune(weights(), 3) == INVALID                            # plain order
+    assert tune(weights(layout=1), 0) == INVALID
 
 
 def test_dense_converter_checks(L):

@@ -137,7 +137,9 @@ def test_bench_line_has_the_contract_keys(monkeypatch, capsys):
     assert line["config"]["workload"] == bench.DEFAULT_WORKLOAD and line["config"]["headline"] == headline
     assert line["config"]["experts"] == 384 and line["config"]["tokens_per_gpu"] == 4096
     assert 0 < line["roofline"]["frac"]
-    assert line["e2e"]["value"] > 0 and line["gpu_launches"] == 20 * (4 + 2 + 3)
+    # routing (4 kernels at T = 4096), quantise, fused gate_up + SwiGLU, down GEMM, combine
+    assert line["e2e"]["value"] > 0 and line["gpu_launches"] == 20 * (4 + 1 + 1 + 1 + 1)
+    assert bench.launches_per_step("layer_unfused", 4096) == 4 + 5
     flops = fake_point(headline)["flops"]
     assert line["value"] == pytest.approx(flops / 0.5e-3 / 1e12)
     assert [e["workload"] for e in line["sweep"]] == points
