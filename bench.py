@@ -77,6 +77,7 @@ for _t in LAYER_T:
     WORKLOADS["kimi_layer_t%d_zipf" % _t] = KIMI + (_t, "zipf", "layer")
 WORKLOADS["kimi_layer_t4096_zipf_unfused"] = KIMI + (4096, "zipf", "layer_unfused")
 WORKLOADS["30b_layer_t256_unfused"] = (128, 8, 2048, 768, 256, "uniform", "layer_unfused")
+WORKLOADS["30b_layer_t4096"] = (128, 8, 2048, 768, 4096, "uniform", "layer")
 # The paper's Table 11 setting (App. D, B200): Kimi gate_up over all 384
 # experts, expert g receiving N * {1, 3/4, 1/2, 1/4}[g % 4] rows, timed as
 # activation quantisation + grouped GEMM (bf16 in, bf16 out); the step is
@@ -341,6 +342,15 @@ def logits_for(routing, seed, T, E):
     return S.zipf_logits_np(seed, T, E) if routing == "zipf" else S.uniform_logits_np(seed, T, E)
 
 
+def parse_gemm_config(text):
+    """'128:296:1,64:296:1' -> {"main": (128, 296, 1), "down": (64, 296, 1)}
+    (the down configuration defaults to the main one)."""
+    parts = [tuple(int(v) for v in p.split(":")) for p in text.split(",")]
+    if not 1 <= len(parts) <= 2 or any(len(p) != 3 for p in parts):
+        raise argparse.ArgumentTypeError("expected TILE_N:NUM_CTAS:SM_MODE[,TILE_N:NUM_CTAS:SM_MODE]")
+    return {"main": parts[0], "down": parts[-1]}
+
+
 def workload_points(name):
     """(points, headline) of a workload name: a sweep or a single workload."""
     if name in SWEEPS:
@@ -430,7 +440,7 @@ def run_cuda(args, rank, world, local_rank):
             out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
 
         # GEMM configurations, frozen by moesq_gemm_autotune after the warm-up
-        # and before the graphs are captured
+        # and before the graphs are captured (or given by --gemm-config)
         tuned = {"main": (0, 0, 0), "down": (0, 0, 0)}
 
         def c_route_quant():
@@ -471,13 +481,17 @@ def run_cuda(args, rank, world, local_rank):
         st, word = m.moesq_get_device_error()
         if st != 0:
             raise RuntimeError("%s: device error word %#x during warm-up" % (name, word))
-        if kind == "layer":
+        if args.gemm_config:
+            tuned["main"] = args.gemm_config["main"]
+            if kind.startswith("layer"):
+                tuned["down"] = args.gemm_config["down"]
+        elif kind == "layer":
             tuned["main"] = m.moesq_gemm_swiglu_autotune(w_main, a_codes, a_scales, rb.rows_cap, rb.counts,
                                                          rb.row_offsets, ga, gh, h_codes, h_scales, reps=3)[0]
         else:
             tuned["main"] = m.moesq_gemm_autotune(w_main, a_codes, a_scales, rb.rows_cap, rb.counts,
                                                   rb.row_offsets, ga, y_main, reps=3)[0]
-        if kind.startswith("layer"):
+        if kind.startswith("layer") and not args.gemm_config:
             tuned["down"] = m.moesq_gemm_autotune(w_dn, h_codes, h_scales, rb.rows_cap, rb.counts,
                                                   rb.row_offsets, gh, y_dn, reps=3)[0]
         step_eager()                          # outputs of the tuned configuration
@@ -865,6 +879,9 @@ def main():
                     choices=sorted(set(WORKLOADS) | set(SWEEPS) | {"tab8_sweep"}))
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gemm-config", default=None, type=parse_gemm_config,
+                    help="TILE_N:NUM_CTAS:SM_MODE of the main GEMM[,of the down GEMM]: fixed configurations "
+                         "instead of the autotuner (profiling runs reproduce the timed launches)")
     args = ap.parse_args()
 
     if "WORLD_SIZE" not in os.environ and args.gpus is not None and args.gpus > 1:
@@ -939,7 +956,8 @@ def main():
                                     "tcgen05.mma.sp kind::mxf4nvf4 on every SM)" % mp)
     tab11_n = r["T"] // 30 if res["headline"].startswith("tab11_") else None
     vs_baseline = value / TAB11[tab11_n][1] if tab11_n else None
-    config.update({"l2": "flushed (256 MiB write) before every step, outside the timed events",
+    config.update({"gemm_config_source": "fixed (--gemm-config)" if args.gemm_config else "moesq autotune",
+                   "l2": "flushed (256 MiB write) before every step, outside the timed events",
                    "timing": "CUDA-graph replay of the step, CUDA events on the launching stream"})
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",

@@ -585,10 +585,15 @@ moesq_status moesq_quantize_act(const uint16_t* x_bf16, int T, int K, const moes
     return MOESQ_ERR_INVALID_ARG;
   }
   cudaStream_t s = as_stream(stream);
-  const int64_t tasks = (int64_t)T * ((K + 1023) / 1024);
+  const int sms = device_info().sms;
+  const int64_t token_tasks = (int64_t)T * ((K + 1023) / 1024);
+  // fewer (token, chunk) tasks than about 16 warps per SM: one warp per slot
+  // instead of one per token, so that enough warps run
+  const int slot_groups = token_tasks < (int64_t)16 * sms ? k : 1;
+  const int64_t tasks = token_tasks * slot_groups;
   if (tasks >= ((int64_t)1 << 31) || (int64_t)T * k >= ((int64_t)1 << 31)) return MOESQ_ERR_UNSUPPORTED_SHAPE;
-  return launch_pdl(quantize_act_kernel, dim3(grid_for(tasks, 8, device_info().sms)), dim3(256), 0, s, x_bf16, T, K,
-                    k, ids, s2r, E, gamma, rows_cap, codes, scales);
+  return launch_pdl(quantize_act_kernel, dim3(grid_for(tasks, 8, sms)), dim3(256), 0, s, x_bf16, T, K, k, ids, s2r,
+                    E, gamma, rows_cap, codes, scales, slot_groups);
 }
 
 moesq_status moesq_act_global_scale(const uint16_t* x_bf16, int64_t n, float* gamma_out, void* stream) {

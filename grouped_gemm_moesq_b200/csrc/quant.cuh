@@ -24,29 +24,34 @@ __device__ __forceinline__ void load32_bf16(const uint16_t* p, float (&v)[32]) {
   }
 }
 
-// One warp task = (token t, 1024-element chunk c of x[t]): lane l loads the
-// scale block [1024 c + 32 l, +32) and takes its amax once, then quantises
-// it for each of the token's k slots with the slot's expert gamma into the
-// slot's row (the fused dispatch + quantisation): the block scale code
-// depends on the slot only through gamma.  Indices stay 32-bit (T * k,
-// rows, K and the task count are below 2^31).  Plain form (slot_to_row ==
-// nullptr): one slot, gamma[0], row = t.
+// One warp task = (token t, 1024-element chunk c of x[t], slot group g):
+// lane l loads the scale block [1024 c + 32 l, +32) and takes its amax once,
+// then quantises it for the token's slots j = g, g + S, ... (S =
+// slot_groups) with the slot's expert gamma into the slot's row (the fused
+// dispatch + quantisation): the block scale code depends on the slot only
+// through gamma.  S = 1 shares one load among all k slots; with few tokens
+// the host splits the slots over S = k warps so that enough warps run.
+// Indices stay 32-bit (T * k * S, rows, K and the task count are below
+// 2^31).  Plain form (slot_to_row == nullptr): one slot, gamma[0], row = t.
 __global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t* __restrict__ x, int T, int K, int k,
                                                            const int32_t* __restrict__ topk_ids,
                                                            const int32_t* __restrict__ slot_to_row, int E,
                                                            const float* __restrict__ gamma, int rows_cap,
-                                                           uint8_t* __restrict__ codes, uint8_t* __restrict__ scales) {
+                                                           uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                                                           int slot_groups) {
   pdl_trigger();
   pdl_wait();
   const int lane = threadIdx.x & 31;
   const int nslots = slot_to_row ? k : 1;
   const int chunks = (K + 1023) >> 10;
-  const int ntasks = T * chunks;
+  const int ntasks = T * chunks * slot_groups;
   const int wstride = gridDim.x * (blockDim.x >> 5);
   const int KB = K / 128;
   for (int task = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); task < ntasks; task += wstride) {
-    const int t = task / chunks;
-    const int k0 = (task - t * chunks) * 1024 + lane * 32;
+    const int grp = task % slot_groups;
+    const int tc = task / slot_groups;
+    const int t = tc / chunks;
+    const int k0 = (tc - t * chunks) * 1024 + lane * 32;
     // lane j < nslots holds slot j's row and gamma (row -1: invalid slot)
     int my_row = -1;
     float my_g = 0.0f;
@@ -57,7 +62,7 @@ __global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t* __res
         if (e >= 0 && e < E && row >= 0 && row < rows_cap) {
           my_row = row;
           my_g = gamma[e];
-        } else if (k0 == lane * 32) {   // reported once per slot (first chunk)
+        } else if (k0 == lane * 32 && lane % slot_groups == grp) {   // once per slot (first chunk)
           record_error(kWhereQuant, kErrFault);
         }
       } else {
@@ -73,7 +78,7 @@ __global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t* __res
 #pragma unroll
       for (int i = 0; i < 32; ++i) a = fmaxf(a, fabsf(v[i]));
     }
-    for (int j = 0; j < nslots; ++j) {
+    for (int j = grp; j < nslots; j += slot_groups) {
       const int row = __shfl_sync(0xffffffffu, my_row, j);
       const float g = __shfl_sync(0xffffffffu, my_g, j);
       if (row < 0 || !act) continue;

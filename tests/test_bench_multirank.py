@@ -172,3 +172,14 @@ def test_tab8_pattern_and_shapes():
     assert set(bench.TAB8) == {"kimi_gate_up", "kimi_down", "30b_gate_up", "30b_down"}
     assert bench.TAB8["kimi_down"][:2] == (7168, 2048) and bench.TAB8["30b_down"][:2] == (2048, 768)
     assert len(bench.TAB8["kimi_gate_up"][2]) * len(bench.TAB8["kimi_gate_up"][3]) == 30
+
+
+def test_gemm_config_flag():
+    """--gemm-config fixes the main (and down) GEMM configuration."""
+    import argparse
+    import bench
+    assert bench.parse_gemm_config("128:296:1") == {"main": (128, 296, 1), "down": (128, 296, 1)}
+    assert bench.parse_gemm_config("128:296:1,64:148:2") == {"main": (128, 296, 1), "down": (64, 148, 2)}
+    for bad in ("128", "128:296", "1:2:3,4:5:6,7:8:9"):
+        with pytest.raises(argparse.ArgumentTypeError):
+            bench.parse_gemm_config(bad)
