@@ -11,6 +11,8 @@
 #include <mutex>
 #include <utility>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/moesq.h"
 #include "common.cuh"
 #include "dense.cuh"
@@ -49,6 +51,16 @@ thread_local cudaError_t t_last_cuda_error = cudaSuccess;
     moesq_status st_ = (call);                             \
     if (st_ != MOESQ_OK) return st_;                       \
   } while (0)
+
+// NVTX range named after the ABI call, around its host-side work (argument
+// checks and launches), for timeline tools; a no-op without a tool attached.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+#define MOESQ_NVTX_RANGE() NvtxRange nvtx_range_(__func__)
 
 inline moesq_status last_launch() {
   const cudaError_t e = cudaGetLastError();
@@ -501,6 +513,7 @@ size_t moesq_weights_bytes(int E, int M, int K, size_t* per_tensor) {
 
 moesq_status moesq_pack_weights(const uint16_t* w_bf16, int e_begin, int e_count, const moesq_weights* out,
                                 void* stream) {
+  MOESQ_NVTX_RANGE();
   MOESQ_TRY(check_weights(out));
   if (!w_bf16 || !aligned(w_bf16, 16)) return MOESQ_ERR_INVALID_ARG;
   if (e_begin < 0 || e_count < 1 || e_begin + e_count > out->E) return MOESQ_ERR_INVALID_ARG;
@@ -524,6 +537,7 @@ moesq_status moesq_pack_weights(const uint16_t* w_bf16, int e_begin, int e_count
 
 moesq_status moesq_import_dense_nvfp4(const uint8_t* codes, const uint8_t* scales, const float* global_scale,
                                       int e_begin, int e_count, const moesq_weights* out, void* stream) {
+  MOESQ_NVTX_RANGE();
   MOESQ_TRY(check_weights(out));
   if (!codes || !scales || !global_scale || !aligned(codes, 16)) return MOESQ_ERR_INVALID_ARG;
   if (e_begin < 0 || e_count < 1 || e_begin + e_count > out->E) return MOESQ_ERR_INVALID_ARG;
@@ -537,6 +551,7 @@ moesq_status moesq_import_dense_nvfp4(const uint8_t* codes, const uint8_t* scale
 }
 
 moesq_status moesq_export_dense_nvfp4(const moesq_weights* w, uint8_t* codes, void* stream) {
+  MOESQ_NVTX_RANGE();
   MOESQ_TRY(check_weights(w));
   if (!codes || !aligned(codes, 16)) return MOESQ_ERR_INVALID_ARG;
   const int64_t n_blocks = (int64_t)w->E * w->M * (w->K / 32);
@@ -559,6 +574,7 @@ size_t moesq_route_workspace_bytes(int T, int E) {
 
 moesq_status moesq_route_permute(const float* logits, const moesq_routing* rt, void* workspace,
                                  size_t workspace_bytes, void* stream) {
+  MOESQ_NVTX_RANGE();
   MOESQ_TRY(check_routing(rt));
   if (!logits) return MOESQ_ERR_INVALID_ARG;
   if (!workspace || workspace_bytes < moesq_route_workspace_bytes(rt->T, rt->E)) return MOESQ_ERR_WORKSPACE;
@@ -567,6 +583,7 @@ moesq_status moesq_route_permute(const float* logits, const moesq_routing* rt, v
 
 moesq_status moesq_quantize_act(const uint16_t* x_bf16, int T, int K, const moesq_routing* rt, const float* gamma,
                                 int rows_cap, uint8_t* codes, uint8_t* scales, void* stream) {
+  MOESQ_NVTX_RANGE();
   if (!x_bf16 || !gamma || !codes || !scales) return MOESQ_ERR_INVALID_ARG;
   if (T < 1 || K < 256 || K % 256) return MOESQ_ERR_UNSUPPORTED_SHAPE;
   if (!aligned(x_bf16, 16) || !aligned(codes, 16)) return MOESQ_ERR_INVALID_ARG;
@@ -597,6 +614,7 @@ moesq_status moesq_quantize_act(const uint16_t* x_bf16, int T, int K, const moes
 }
 
 moesq_status moesq_act_global_scale(const uint16_t* x_bf16, int64_t n, float* gamma_out, void* stream) {
+  MOESQ_NVTX_RANGE();
   if (!x_bf16 || !gamma_out || n < 1) return MOESQ_ERR_INVALID_ARG;
   cudaStream_t s = as_stream(stream);
   MOESQ_CUDA(cudaMemsetAsync(gamma_out, 0, sizeof(float), s));
@@ -611,6 +629,7 @@ moesq_status moesq_grouped_sparse_gemm(const moesq_weights* w, const uint8_t* a_
                                        int rows_cap, const int32_t* counts, const int32_t* row_offsets,
                                        const float* gamma_a, uint16_t* y_bf16, const moesq_gemm_config* cfg,
                                        void* stream) {
+  MOESQ_NVTX_RANGE();
   MOESQ_TRY(check_weights(w));
   if (!a_codes || !a_scales || !counts || !row_offsets || !gamma_a || !y_bf16) return MOESQ_ERR_INVALID_ARG;
   if (rows_cap < 128 || rows_cap % 128) return MOESQ_ERR_INVALID_ARG;
@@ -642,6 +661,7 @@ moesq_status moesq_grouped_dense_gemm(const moesq_dense_weights* w, const uint8_
                                       const uint8_t* a_scales16, int rows_cap, const int32_t* counts,
                                       const int32_t* row_offsets, const float* gamma_a, uint16_t* y_bf16,
                                       const moesq_gemm_config* cfg, void* stream) {
+  MOESQ_NVTX_RANGE();
   MOESQ_TRY(check_dense_weights(w));
   if (!a_codes || !a_scales16 || !counts || !row_offsets || !gamma_a || !y_bf16) return MOESQ_ERR_INVALID_ARG;
   if (rows_cap < 128 || rows_cap % 128) return MOESQ_ERR_INVALID_ARG;
@@ -679,6 +699,7 @@ size_t moesq_dense_weights_bytes(int E, int M, int K, size_t* per_tensor) {
 
 moesq_status moesq_pack_dense_nvfp4(const uint16_t* w_bf16, int e_begin, int e_count, const moesq_dense_weights* out,
                                     void* stream) {
+  MOESQ_NVTX_RANGE();
   MOESQ_TRY(check_dense_weights(out));
   if (!w_bf16 || !aligned(w_bf16, 16)) return MOESQ_ERR_INVALID_ARG;
   if (e_begin < 0 || e_count < 1 || e_begin + e_count > out->E) return MOESQ_ERR_INVALID_ARG;
@@ -700,6 +721,7 @@ moesq_status moesq_pack_dense_nvfp4(const uint16_t* w_bf16, int e_begin, int e_c
 }
 
 moesq_status moesq_expand_scales16(const uint8_t* a_scales, int rows_cap, int K, uint8_t* a_scales16, void* stream) {
+  MOESQ_NVTX_RANGE();
   if (!a_scales || !a_scales16 || !aligned(a_scales, 4) || !aligned(a_scales16, 4)) return MOESQ_ERR_INVALID_ARG;
   if (rows_cap < 128 || rows_cap % 128 || K < 256 || K % 256) return MOESQ_ERR_UNSUPPORTED_SHAPE;
   const int64_t n_words = (int64_t)rows_cap * (K / 16) / 4;
@@ -759,6 +781,7 @@ moesq_status moesq_gemm_autotune(const moesq_weights* w, const uint8_t* a_codes,
                                  int rows_cap, const int32_t* counts, const int32_t* row_offsets,
                                  const float* gamma_a, uint16_t* y_bf16, int reps,
                                  moesq_gemm_config* best, float* best_ms, void* stream) {
+  MOESQ_NVTX_RANGE();
   MOESQ_TRY(check_weights(w));
   if (!best || !best_ms || reps < 1) return MOESQ_ERR_INVALID_ARG;
   cudaStream_t s = as_stream(stream);
@@ -779,6 +802,7 @@ moesq_status moesq_grouped_sparse_gemm_swiglu(const moesq_weights* w, const uint
                                               const int32_t* row_offsets, const float* gamma_a,
                                               const float* gamma_h, uint8_t* h_codes, uint8_t* h_scales,
                                               const moesq_gemm_config* cfg, void* stream) {
+  MOESQ_NVTX_RANGE();
   MOESQ_TRY(check_weights(w));
   if (w->layout != MOESQ_LAYOUT_SWIGLU) return MOESQ_ERR_INVALID_ARG;
   if (!a_codes || !a_scales || !counts || !row_offsets || !gamma_a || !gamma_h || !h_codes || !h_scales)
@@ -809,6 +833,7 @@ moesq_status moesq_gemm_swiglu_autotune(const moesq_weights* w, const uint8_t* a
                                         const float* gamma_a, const float* gamma_h, uint8_t* h_codes,
                                         uint8_t* h_scales, int reps, moesq_gemm_config* best, float* best_ms,
                                         void* stream) {
+  MOESQ_NVTX_RANGE();
   MOESQ_TRY(check_weights(w));
   if (w->layout != MOESQ_LAYOUT_SWIGLU) return MOESQ_ERR_INVALID_ARG;
   if (!best || !best_ms || reps < 1) return MOESQ_ERR_INVALID_ARG;
@@ -826,6 +851,7 @@ moesq_status moesq_gemm_swiglu_autotune(const moesq_weights* w, const uint8_t* a
 
 moesq_status moesq_swiglu_quant(const uint16_t* y_gu, int I, const moesq_routing* rt, const float* gamma_h,
                                 uint8_t* h_codes, uint8_t* h_scales, int gu_layout, void* stream) {
+  MOESQ_NVTX_RANGE();
   MOESQ_TRY(check_routing(rt));
   if (!y_gu || !gamma_h || !h_codes || !h_scales) return MOESQ_ERR_INVALID_ARG;
   if (gu_layout != MOESQ_LAYOUT_PLAIN && gu_layout != MOESQ_LAYOUT_SWIGLU) return MOESQ_ERR_INVALID_ARG;
@@ -838,6 +864,7 @@ moesq_status moesq_swiglu_quant(const uint16_t* y_gu, int I, const moesq_routing
 }
 
 moesq_status moesq_combine(const uint16_t* y, int H, const moesq_routing* rt, uint16_t* out, void* stream) {
+  MOESQ_NVTX_RANGE();
   MOESQ_TRY(check_routing(rt));
   if (!y || !out || H < 8 || H % 8) return MOESQ_ERR_INVALID_ARG;
   if (!aligned(y, 16) || !aligned(out, 16)) return MOESQ_ERR_INVALID_ARG;
@@ -865,6 +892,7 @@ size_t moesq_layer_host_workspace_bytes(int T, int k, int E, int H, int I) {
 moesq_status moesq_moe_layer(const uint16_t* x_bf16, const float* logits, int T, int k, const moesq_weights* w_gu,
                              const moesq_weights* w_dn, const float* gamma_a_gu, const float* gamma_a_dn,
                              uint16_t* out_bf16, void* workspace, size_t workspace_bytes, void* stream) {
+  MOESQ_NVTX_RANGE();
   MOESQ_TRY(check_layer(T, k, w_gu, w_dn));
   if (!x_bf16 || !logits || !gamma_a_gu || !gamma_a_dn || !out_bf16) return MOESQ_ERR_INVALID_ARG;
   const int E = w_gu->E, H = w_gu->K, I = w_gu->M / 2;
@@ -878,6 +906,7 @@ moesq_status moesq_moe_layer_host(const uint16_t* x_bf16_host, const float* logi
                                   const moesq_weights* w_gu, const moesq_weights* w_dn, const float* gamma_a_gu,
                                   const float* gamma_a_dn, uint16_t* out_bf16_host, void* workspace,
                                   size_t workspace_bytes, void* stream) {
+  MOESQ_NVTX_RANGE();
   MOESQ_TRY(check_layer(T, k, w_gu, w_dn));
   if (!x_bf16_host || !logits_host || !gamma_a_gu || !gamma_a_dn || !out_bf16_host) return MOESQ_ERR_INVALID_ARG;
   const int E = w_gu->E, H = w_gu->K, I = w_gu->M / 2;
@@ -896,6 +925,7 @@ moesq_status moesq_moe_layer_host(const uint16_t* x_bf16_host, const float* logi
 moesq_status moesq_calibrate_layer(const uint16_t* x_bf16, const float* logits, int T, int k,
                                    const moesq_weights* w_gu, const moesq_weights* w_dn, float* gamma_a_gu,
                                    float* gamma_a_dn, void* workspace, size_t workspace_bytes, void* stream) {
+  MOESQ_NVTX_RANGE();
   MOESQ_TRY(check_layer(T, k, w_gu, w_dn));
   if (!x_bf16 || !logits || !gamma_a_gu || !gamma_a_dn) return MOESQ_ERR_INVALID_ARG;
   const int E = w_gu->E, H = w_gu->K, I = w_gu->M / 2;
@@ -932,6 +962,7 @@ moesq_status moesq_debug_bounded_wait(uint64_t timeout_ns, void* stream) {
 
 moesq_status moesq_mma_peak(int sparse, int n, int ctas_per_sm, int with_copies, int iters, double* tflops,
                             void* stream) {
+  MOESQ_NVTX_RANGE();
   if (!tflops || iters < 1 || (sparse != 0 && sparse != 1)) return MOESQ_ERR_INVALID_ARG;
   if (with_copies != 0 && with_copies != 1) return MOESQ_ERR_INVALID_ARG;
   if (ctas_per_sm != 1 && ctas_per_sm != 2) return MOESQ_ERR_INVALID_ARG;
@@ -971,6 +1002,7 @@ moesq_status moesq_mma_peak(int sparse, int n, int ctas_per_sm, int with_copies,
 }
 
 moesq_status moesq_route_permute_noalloc(const float* logits, const moesq_routing* rt, void* stream) {
+  MOESQ_NVTX_RANGE();
   MOESQ_TRY(check_routing(rt));
   if (!logits) return MOESQ_ERR_INVALID_ARG;
   if (rt->T > kNoAllocMaxT) return MOESQ_ERR_UNSUPPORTED_SHAPE;   // beyond the static scratch

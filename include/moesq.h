@@ -15,8 +15,10 @@
  *    void*, NULL = the legacy default stream), does no host synchronisation
  *    and reads no device data on the host, so a sequence of calls can be
  *    captured into a CUDA graph.  The exceptions are moesq_get_device_error
- *    (synchronises), moesq_moe_layer_host (synchronises at the end) and
- *    moesq_gemm_autotune (times launches, synchronises).
+ *    (synchronises), moesq_moe_layer_host (synchronises at the end), the
+ *    autotuners and moesq_mma_peak (time launches, synchronise).
+ *  - Every call that launches work opens an NVTX range named after itself
+ *    (host side, around its checks and launches) for timeline tools.
  *  - Shape and argument errors are detected on the host and returned at once;
  *    nothing is launched then.  Faults detected on the device (inconsistent
  *    routing counts, out-of-range expert ids, a bounded wait that ran out)
