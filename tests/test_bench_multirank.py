@@ -183,3 +183,29 @@ def test_gemm_config_flag():
     for bad in ("128", "128:296", "1:2:3,4:5:6,7:8:9"):
         with pytest.raises(argparse.ArgumentTypeError):
             bench.parse_gemm_config(bad)
+
+
+def test_step_work_algorithmic_bytes():
+    """The per-GEMM algorithmic bytes the roofline divides by: packed weights
+    of the touched experts (11 M K / 32 each), the
+    NVFP4 activation rows in (K/2 codes + K/32 scales per row) and the
+    output: bf16 rows, or for the fused layer the requantised h rows."""
+    import bench
+    from grouped_gemm_moesq_b200.metrics import packed_weight_bytes
+    E, k, H, I, T = 8, 2, 512, 256, 64
+    counts = np.array([10, 0, 30, 5, 0, 40, 20, 23])
+    R = T * k
+    assert packed_weight_bytes(2 * I, H) == 11 * 2 * I * H // 32
+    fl, wb, gb, gf = bench.step_work(E, k, H, I, T, counts, "layer")
+    touched = 6
+    gu_w, dn_w = touched * packed_weight_bytes(2 * I, H), touched * packed_weight_bytes(H, I)
+    assert wb == gu_w + dn_w
+    assert gb["gate_up"] == gu_w + R * (H // 2 + H // 32) + R * (I // 2 + I // 32)      # fused: h out
+    assert gb["down"] == dn_w + R * (I // 2 + I // 32) + R * H * 2
+    assert gf["gate_up"] == 2.0 * 2 * I * H * R and gf["down"] == 2.0 * H * I * R and fl == gf["gate_up"] + gf["down"]
+    _, _, gb_u, _ = bench.step_work(E, k, H, I, T, counts, "layer_unfused")
+    assert gb_u["gate_up"] == gu_w + R * (H // 2 + H // 32) + R * 2 * I * 2             # unfused: bf16 y_gu out
+    _, _, gb_q, gf_q = bench.step_work(E, k, H, I, T, counts, "quant_gemm")
+    Rq = int(counts.sum())                                                               # fixed grouping: routed rows
+    assert gb_q == {"gate_up": gu_w + Rq * (H // 2 + H // 32) + Rq * 2 * I * 2}
+    assert gf_q == {"gate_up": 2.0 * 2 * I * H * Rq}
