@@ -808,7 +808,8 @@ moesq_status moesq_grouped_sparse_gemm_swiglu(const moesq_weights* w, const uint
   if (!a_codes || !a_scales || !counts || !row_offsets || !gamma_a || !gamma_h || !h_codes || !h_scales)
     return MOESQ_ERR_INVALID_ARG;
   if (rows_cap < 128 || rows_cap % 128) return MOESQ_ERR_INVALID_ARG;
-  if (!aligned(a_codes, 16) || !aligned(a_scales, 16)) return MOESQ_ERR_INVALID_ARG;
+  // 16-byte code stores per (row, 32-feature block) in the epilogue
+  if (!aligned(a_codes, 16) || !aligned(a_scales, 16) || !aligned(h_codes, 16)) return MOESQ_ERR_INVALID_ARG;
   int tile_n = cfg ? cfg->tile_n : 0;
   const int num_ctas = cfg ? cfg->num_ctas : 0;
   const int sm_mode = cfg ? cfg->sm_mode : 0;

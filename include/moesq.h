@@ -394,8 +394,8 @@ moesq_status moesq_swiglu_quant(const uint16_t* y_gu, int I, const moesq_routing
  * row).  The bf16 gate_up output never reaches memory.  Same row space,
  * validation and cfg as moesq_grouped_sparse_gemm, except that sm_mode 2
  * is not offered (MOESQ_ERR_UNSUPPORTED_SHAPE) and weights of another
- * layout are rejected (MOESQ_ERR_INVALID_ARG).  a_codes and a_scales are
- * 16-byte aligned. */
+ * layout are rejected (MOESQ_ERR_INVALID_ARG).  a_codes, a_scales and
+ * h_codes are 16-byte aligned. */
 moesq_status moesq_grouped_sparse_gemm_swiglu(const moesq_weights* w, const uint8_t* a_codes,
                                               const uint8_t* a_scales, int rows_cap, const int32_t* counts,
                                               const int32_t* row_offsets, const float* gamma_a,

@@ -136,6 +136,7 @@ def test_weight_layout_and_fused_gemm_checks(L):
     assert fused(weights()) == INVALID                              # plain order: not a fused gate_up stack
     assert fused(weights(layout=1), h_codes=None) == INVALID
     assert fused(weights(layout=1), a_scales=ptr(8)) == INVALID
+    assert fused(weights(layout=1), h_codes=ptr(8)) == INVALID      # 16-byte code stores
     assert fused(weights(layout=1), B.moesq_gemm_config(96, 0, 0)) == INVALID
     assert fused(weights(layout=1), B.moesq_gemm_config(128, 0, 2)) == SHAPE   # no SM-pair form
     best, ms = B.moesq_gemm_config(0, 0, 0), ctypes.c_float(0)
