@@ -163,6 +163,10 @@ moesq_status check_routing(const moesq_routing* rt) {
   if (!rt->topk_ids || !rt->topk_w || !rt->counts || !rt->offsets || !rt->row_offsets || !rt->sorted_to_slot ||
       !rt->slot_to_row)
     return MOESQ_ERR_INVALID_ARG;
+  const void* arrays[7] = {rt->topk_ids, rt->topk_w, rt->counts, rt->offsets, rt->row_offsets, rt->sorted_to_slot,
+                           rt->slot_to_row};
+  for (const void* a : arrays)
+    if (!aligned(a, 4)) return MOESQ_ERR_INVALID_ARG;
   if (rt->rows_cap % 128 || rt->rows_cap < moesq_rows_capacity(rt->T, rt->k, rt->E)) return MOESQ_ERR_INVALID_ARG;
   return MOESQ_OK;
 }
@@ -576,8 +580,9 @@ moesq_status moesq_route_permute(const float* logits, const moesq_routing* rt, v
                                  size_t workspace_bytes, void* stream) {
   MOESQ_NVTX_RANGE();
   MOESQ_TRY(check_routing(rt));
-  if (!logits) return MOESQ_ERR_INVALID_ARG;
+  if (!logits || !aligned(logits, 4)) return MOESQ_ERR_INVALID_ARG;
   if (!workspace || workspace_bytes < moesq_route_workspace_bytes(rt->T, rt->E)) return MOESQ_ERR_WORKSPACE;
+  if (!aligned(workspace, 4)) return MOESQ_ERR_INVALID_ARG;
   return route_launch(logits, rt, static_cast<int32_t*>(workspace), as_stream(stream));
 }
 
@@ -586,7 +591,7 @@ moesq_status moesq_quantize_act(const uint16_t* x_bf16, int T, int K, const moes
   MOESQ_NVTX_RANGE();
   if (!x_bf16 || !gamma || !codes || !scales) return MOESQ_ERR_INVALID_ARG;
   if (T < 1 || K < 256 || K % 256) return MOESQ_ERR_UNSUPPORTED_SHAPE;
-  if (!aligned(x_bf16, 16) || !aligned(codes, 16)) return MOESQ_ERR_INVALID_ARG;
+  if (!aligned(x_bf16, 16) || !aligned(codes, 16) || !aligned(gamma, 4)) return MOESQ_ERR_INVALID_ARG;
   if (rows_cap < 128 || rows_cap % 128) return MOESQ_ERR_INVALID_ARG;
   int k = 1, E = 1;
   const int32_t* ids = nullptr;
@@ -634,6 +639,7 @@ moesq_status moesq_grouped_sparse_gemm(const moesq_weights* w, const uint8_t* a_
   if (!a_codes || !a_scales || !counts || !row_offsets || !gamma_a || !y_bf16) return MOESQ_ERR_INVALID_ARG;
   if (rows_cap < 128 || rows_cap % 128) return MOESQ_ERR_INVALID_ARG;
   if (!aligned(a_codes, 16) || !aligned(a_scales, 16) || !aligned(y_bf16, 2)) return MOESQ_ERR_INVALID_ARG;
+  if (!aligned(counts, 4) || !aligned(row_offsets, 4) || !aligned(gamma_a, 4)) return MOESQ_ERR_INVALID_ARG;
   int tile_n = cfg ? cfg->tile_n : 0;
   const int num_ctas = cfg ? cfg->num_ctas : 0;
   const int sm_mode = cfg ? cfg->sm_mode : 0;
@@ -666,6 +672,7 @@ moesq_status moesq_grouped_dense_gemm(const moesq_dense_weights* w, const uint8_
   if (!a_codes || !a_scales16 || !counts || !row_offsets || !gamma_a || !y_bf16) return MOESQ_ERR_INVALID_ARG;
   if (rows_cap < 128 || rows_cap % 128) return MOESQ_ERR_INVALID_ARG;
   if (!aligned(a_codes, 16) || !aligned(a_scales16, 16) || !aligned(y_bf16, 2)) return MOESQ_ERR_INVALID_ARG;
+  if (!aligned(counts, 4) || !aligned(row_offsets, 4) || !aligned(gamma_a, 4)) return MOESQ_ERR_INVALID_ARG;
   int tile_n = cfg ? cfg->tile_n : 0;
   const int num_ctas = cfg ? cfg->num_ctas : 0;
   const int sm_mode = cfg ? cfg->sm_mode : 0;
@@ -807,6 +814,8 @@ moesq_status moesq_grouped_sparse_gemm_swiglu(const moesq_weights* w, const uint
   if (w->layout != MOESQ_LAYOUT_SWIGLU) return MOESQ_ERR_INVALID_ARG;
   if (!a_codes || !a_scales || !counts || !row_offsets || !gamma_a || !gamma_h || !h_codes || !h_scales)
     return MOESQ_ERR_INVALID_ARG;
+  if (!aligned(counts, 4) || !aligned(row_offsets, 4) || !aligned(gamma_a, 4) || !aligned(gamma_h, 4))
+    return MOESQ_ERR_INVALID_ARG;
   if (rows_cap < 128 || rows_cap % 128) return MOESQ_ERR_INVALID_ARG;
   // 16-byte code stores per (row, 32-feature block) in the epilogue
   if (!aligned(a_codes, 16) || !aligned(a_scales, 16) || !aligned(h_codes, 16)) return MOESQ_ERR_INVALID_ARG;
@@ -854,7 +863,7 @@ moesq_status moesq_swiglu_quant(const uint16_t* y_gu, int I, const moesq_routing
                                 uint8_t* h_codes, uint8_t* h_scales, int gu_layout, void* stream) {
   MOESQ_NVTX_RANGE();
   MOESQ_TRY(check_routing(rt));
-  if (!y_gu || !gamma_h || !h_codes || !h_scales) return MOESQ_ERR_INVALID_ARG;
+  if (!y_gu || !gamma_h || !h_codes || !h_scales || !aligned(gamma_h, 4)) return MOESQ_ERR_INVALID_ARG;
   if (gu_layout != MOESQ_LAYOUT_PLAIN && gu_layout != MOESQ_LAYOUT_SWIGLU) return MOESQ_ERR_INVALID_ARG;
   if (I < 256 || I % 256) return MOESQ_ERR_UNSUPPORTED_SHAPE;
   if (!aligned(y_gu, 16) || !aligned(h_codes, 16)) return MOESQ_ERR_INVALID_ARG;
@@ -1005,7 +1014,7 @@ moesq_status moesq_mma_peak(int sparse, int n, int ctas_per_sm, int with_copies,
 moesq_status moesq_route_permute_noalloc(const float* logits, const moesq_routing* rt, void* stream) {
   MOESQ_NVTX_RANGE();
   MOESQ_TRY(check_routing(rt));
-  if (!logits) return MOESQ_ERR_INVALID_ARG;
+  if (!logits || !aligned(logits, 4)) return MOESQ_ERR_INVALID_ARG;
   if (rt->T > kNoAllocMaxT) return MOESQ_ERR_UNSUPPORTED_SHAPE;   // beyond the static scratch
   const int nblk = (rt->T + kRouteTPB - 1) / kRouteTPB;
   if ((size_t)nblk * (size_t)rt->E > kNoAllocScratchInts) return MOESQ_ERR_UNSUPPORTED_SHAPE;

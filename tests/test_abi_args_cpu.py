@@ -96,6 +96,23 @@ def test_routing_checks(L):
     assert L.moesq_route_permute_noalloc(ptr(), ctypes.byref(routing(T=16385, E=8, k=2)), None) == SHAPE
 
 
+def test_misaligned_index_arrays_are_refused(L):
+    """Arrays read with 4-byte loads (routing, counts, global scales) must be
+    4-byte aligned; the calls refuse them on the host."""
+    for field in ("topk_ids", "topk_w", "counts", "offsets", "row_offsets", "sorted_to_slot", "slot_to_row"):
+        rt = routing(**{field: P + 2})
+        assert L.moesq_route_permute(ptr(), ctypes.byref(rt), ptr(), 1 << 20, None) == INVALID, field
+    rt = routing()
+    assert L.moesq_route_permute(ptr(2), ctypes.byref(rt), ptr(), 1 << 20, None) == INVALID        # logits
+    assert L.moesq_route_permute(ptr(), ctypes.byref(rt), ptr(2), 1 << 20, None) == INVALID        # workspace
+    assert L.moesq_route_permute_noalloc(ptr(2), ctypes.byref(rt), None) == INVALID
+    assert gemm(L, weights(), counts=ptr(2)) == INVALID
+    assert gemm(L, weights(), row_offsets=ptr(2)) == INVALID
+    assert gemm(L, weights(), gamma=ptr(2)) == INVALID
+    assert L.moesq_quantize_act(ptr(), 8, 512, ctypes.byref(rt), ptr(2), rt.rows_cap, ptr(), ptr(), None) == INVALID
+    assert L.moesq_swiglu_quant(ptr(), 256, ctypes.byref(rt), ptr(2), ptr(), ptr(), 0, None) == INVALID
+
+
 def test_quantise_swiglu_combine_checks(L):
     rt = routing()
     rc = rt.rows_cap
