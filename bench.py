@@ -5,7 +5,7 @@ dispatch-quantise, gate_up grouped sparse GEMM, SwiGLU + requantise, down
 grouped sparse GEMM, router-weighted combine (weight packing is offline and
 not timed).  The default workload is the Kimi-K2.5-shaped MoE layer (384
 experts, top-8, hidden 7168, intermediate 2048 -> gate_up N = 4096) swept over
-T = 1 ... 16384 tokens with uniform and Zipf(1.1) routing; the headline
+T = 1, 4, 16, ..., 16384 tokens with uniform and Zipf(1.1) routing; the headline
 numbers are those of T = 4096 with Zipf routing, and every point of the sweep
 is in `sweep`.  Synthetic data of the pages' distributions.
 
@@ -50,7 +50,7 @@ from grouped_gemm_moesq_b200.metrics import packed_weight_bytes  # noqa: E402
 METRIC = "paired-4:8 NVFP4 grouped GEMM TFLOP/s + weight GB/s vs roofline, per token count"
 
 KIMI = (384, 8, 7168, 2048)        # experts, top-k, hidden, intermediate
-LAYER_T = (1, 16, 64, 256, 1024, 4096, 16384)
+LAYER_T = (1, 4, 16, 64, 256, 1024, 4096, 16384)
 
 # name -> (E, k, H, I, T, routing, kind).  kind: "layer" (the whole path,
 # SwiGLU + requantisation fused into the gate_up GEMM), "layer_unfused" (the
@@ -109,6 +109,8 @@ TAB8 = {
     "30b_down": (2048, 768, (16, 32, 64, 128, 256, 512, 1024), (8, 16, 32, 64, 128)),
 }
 
+SPEC_HBM_GBS = 8000.0       # B200 HBM3e specification (8 TB/s), beside the measured copy rate
+PAPER_SPARSE_FP4_TFLOPS = 18000.0   # the pages' sparse FP4 tensor peak, dense-equivalent
 FP4_OVER_BF16 = 4.0    # nominal dense tensor-core ratio, fp4 : bf16 (9 : 2.25 PFLOP/s)
 SPARSE_FACTOR = 2.0    # a structured-sparse MMA runs the dense-equivalent contraction at twice the rate
 
@@ -172,6 +174,8 @@ def gemm_roofline(gbytes, gfl, gemm_ms, peaks, traffic, gname):
     roofline.update({"traffic": traffic, "algorithmic_bytes": gbytes, "dense_equiv_flops": gfl,
                      "kernel": "grouped_sparse_gemm (%s)" % gname, "kernel_ms": gemm_ms,
                      "hbm_frac": hbm_ach / hbm_peak, "tensor_frac": tc_ach / tc_peak,
+                     "hbm_frac_of_spec": hbm_ach / SPEC_HBM_GBS,
+                     "tensor_frac_of_paper_peak": tc_ach / PAPER_SPARSE_FP4_TFLOPS,
                      "peak_source": "%s (tensor peak = dense bf16 burst x %g fp4/bf16 x %g sparse)"
                      % (peaks["source"], FP4_OVER_BF16, SPARSE_FACTOR)})
     return roofline

@@ -109,7 +109,7 @@ def test_bench_line_has_the_contract_keys(monkeypatch, capsys):
     import sys
     import bench
     points, headline = bench.workload_points(bench.DEFAULT_WORKLOAD)
-    assert headline in points and len(points) == 14
+    assert headline in points and len(points) == 16
 
     def fake_point(name):
         E, k, H, I, T, routing, kind = bench.WORKLOADS[name]
