@@ -27,7 +27,11 @@
 //           i overlaps the main loop of tile i+1; with 128-row tiles the other
 //           CTA covers the epilogue.
 //   warps 2-5 epilogue: tcgen05.ld of the fp32 accumulator, times alpha_e,
-//           rounded to bf16 and stored for the valid rows only.
+//           rounded to bf16 and stored for the valid rows only; or, for a
+//           gate_up stack in the SwiGLU kernel row order (SWIGLU), h =
+//           SiLU(gate) * up requantised to NVFP4 (App. D.1 "fused SwiGLU
+//           with requantization"), so that the bf16 gate_up output never
+//           reaches memory.
 // Work units are (expert, 128-row weight block, TN-row token block); the
 // per-expert token counts stay on the device and every CTA derives the unit
 // list from them (no host synchronisation).  Units are taken round-robin;
