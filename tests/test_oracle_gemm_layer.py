@@ -126,6 +126,32 @@ def test_layer_single_expert_chain():
     assert np.abs(got - ref).max() / np.abs(ref).max() < 1e-2
 
 
+def test_layer_identical_experts_reduce_to_weighted_single_expert():
+    """E identical experts with equal global scales compute the same function
+    of a token, so routing, dispatch, grouped GEMMs and combine must give
+    out[t] = bf16((sum_j w_tj) * y[t]), y[t] the single-expert layer's output
+    row (exact in bf16), for every token: a token row landing in another
+    token's slot, a dropped or doubled slot, or a wrong router weight breaks
+    it."""
+    E, k, H, I, T = 6, 3, 128, 64, 16
+    w1gu = S.expert_weights_bf16_np(9, 0, 0, 2 * I, H)[None]
+    w1dn = S.expert_weights_bf16_np(9, 1, 0, H, I)[None]
+    p1gu, p1dn = O.pack_weights(w1gu), O.pack_weights(w1dn)
+    pEgu, pEdn = O.pack_weights(np.repeat(w1gu, E, axis=0)), O.pack_weights(np.repeat(w1dn, E, axis=0))
+    x = S.activations_bf16_np(9, T, H)
+    ga1 = np.array([O.act_global_scale(x)], np.float32)
+    _, st = O.moe_layer(x, np.zeros((T, 1), np.float32), 1, p1gu, p1dn, ga1, np.ones(1, np.float32), keep=True)
+    gh1 = np.array([O.global_scale(np.abs(st["h"]).max())], np.float32)
+    y1 = O.moe_layer(x, np.zeros((T, 1), np.float32), 1, p1gu, p1dn, ga1, gh1)
+    logits = S.uniform_logits_np(9, T, E)
+    outE = O.moe_layer(x, logits, k, pEgu, pEdn, np.repeat(ga1, E), np.repeat(gh1, E))
+    wsum = O.route(logits, k).topk_w.reshape(T, k).astype(np.float64).sum(axis=1)
+    y1f = S.bf16_bits_to_f32_np(y1).astype(np.float64)
+    want = np.array([[O.bf16_round(wsum[t] * y1f[t, h]) for h in range(H)] for t in range(T)], np.uint16)
+    assert (wsum > 0.3).all() and (wsum <= 1.0 + 1e-6).all()
+    assert (outE == want).all()
+
+
 def test_effective_tflops_formula_table10():
     """App. D.2's TFLOP/s_eff with Table 10's setting reproduces the printed
     2627 TFLOP/s from the printed 0.687 ms (to the printed precision)."""
