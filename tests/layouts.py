@@ -158,3 +158,13 @@ def scales32_to_scales16_mma(scales32: np.ndarray) -> np.ndarray:
     """Row-major per-32 scales [R, K/32] -> per-16 scales (each twice) in the
     dense MMA layout (flat)."""
     return scales_to_mma(np.repeat(scales32, 2, axis=1))
+
+
+def swiglu_kernel_rows(M: int) -> np.ndarray:
+    """perm[p] = storage row held by kernel row p in the SwiGLU order: block
+    b of 128 kernel rows = gate rows 64 b + [0, 64), then up rows
+    M/2 + 64 b + [0, 64)."""
+    I = M // 2
+    p = np.arange(M)
+    b, r = p // 128, p % 128
+    return np.where(r < 64, 64 * b + r, I + 64 * b + r - 64)

@@ -19,27 +19,9 @@ import layouts as L
 import oracle as O
 import synthetic as S
 from gpu_cases import requant_mismatches, to_dev, to_np, weights_np
+from layouts import swiglu_kernel_rows
 
 pytestmark = pytest.mark.gpu
-
-
-def swiglu_kernel_rows(M: int) -> np.ndarray:
-    """perm[p] = storage row held by kernel row p in the SwiGLU order: block
-    b of 128 kernel rows = gate rows 64 b + [0, 64), then up rows
-    M/2 + 64 b + [0, 64)."""
-    I = M // 2
-    p = np.arange(M)
-    b, r = p // 128, p % 128
-    return np.where(r < 64, 64 * b + r, I + 64 * b + r - 64)
-
-
-def test_swiglu_order_is_a_pairing_permutation():
-    perm = swiglu_kernel_rows(1536)
-    assert sorted(perm.tolist()) == list(range(1536))
-    # kernel rows 128 b + j and 128 b + 64 + j hold gate and up of feature 64 b + j
-    for b in range(12):
-        for j in (0, 17, 63):
-            assert perm[128 * b + j] == 64 * b + j and perm[128 * b + 64 + j] == 768 + 64 * b + j
 
 
 def test_pack_swiglu_layout(cuda_lib):

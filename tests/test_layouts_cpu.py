@@ -71,3 +71,12 @@ def test_dense_tile_layout_round_trip_and_swizzle():
     s32 = rng.integers(0, 127, size=(128, K // 32), dtype=np.uint8)
     s16 = L.mma_to_scales(L.scales32_to_scales16_mma(s32), 128, 2 * K)
     assert (s16[:, 0::2] == s32).all() and (s16[:, 1::2] == s32).all()
+
+
+def test_swiglu_order_is_a_pairing_permutation():
+    perm = L.swiglu_kernel_rows(1536)
+    assert sorted(perm.tolist()) == list(range(1536))
+    # kernel rows 128 b + j and 128 b + 64 + j hold gate and up of feature 64 b + j
+    for b in range(12):
+        for j in (0, 17, 63):
+            assert perm[128 * b + j] == 64 * b + j and perm[128 * b + 64 + j] == 768 + 64 * b + j
